@@ -1,0 +1,178 @@
+/*
+ * wise.h -- C ABI of the WISE attention hot path on NVIDIA B200 (sm_100a).
+ *
+ * WISE ("Working-set Inference with Support Exploitation") is described in
+ * Wan & Chen, "Attention Routing Stabilizes Early: Working-Set Inference for
+ * Recurrent-Depth Language Models" (arXiv 2609.27373), "the WISE paper"
+ * below.  One recurrent step of one attention layer goes through:
+ *
+ *   exploration steps t <= t_d : wise_full_attn_mass   (dense causal attention,
+ *                                  plus block mass on discovery-window steps)
+ *                                wise_select_union     (cumulative-eta support,
+ *                                  OR-ed into the working set)
+ *   once, after step t_d       : wise_build_schedule   (CSR key-block schedule)
+ *   late steps t > t_d         : wise_sparse_attn      (block-sparse attention)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Block size B = 32 tokens (WISE paper section 7.1, "WISE configuration").
+ * - Q, K, V, O are bf16, contiguous [batch, heads, seqlen, head_dim]
+ *   (row-major, head_dim fastest).  head_dim is 64, 96 or 128; seqlen is a
+ *   positive multiple of 32 and at most 16384.  nq = seqlen / 32 blocks.
+ *   "BH" = batch * heads.  Q, K, V, O base addresses must be 16-byte aligned.
+ * - All data pointers are DEVICE pointers allocated by the caller; the library
+ *   allocates no device memory and never takes ownership.  Host pointers are
+ *   marked as such.
+ * - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *   enqueue work and return; the one exception is wise_build_schedule with a
+ *   non-NULL nnz_out, which synchronises `stream`.
+ * - Return value: WISE_OK (0) on success, a negative WISE_ERR_* otherwise.
+ *   On error nothing is enqueued and wise_last_error() (thread-local) holds a
+ *   message.  Faults detected on the device (an invalid schedule entry, or a
+ *   pipeline wait that ran out of time) do not stop the kernel: they set bits
+ *   in a device status word read by wise_device_status().
+ */
+#ifndef WISE_H_
+#define WISE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define WISE_OK 0
+#define WISE_ERR_ARG (-1)      /* NULL pointer where one is required, bad eta */
+#define WISE_ERR_SHAPE (-2)    /* unsupported head_dim / seqlen / sizes        */
+#define WISE_ERR_ALIGN (-3)    /* pointer not 16-byte aligned                  */
+#define WISE_ERR_CAPACITY (-4) /* col_idx too small for the schedule           */
+#define WISE_ERR_CUDA (-5)     /* CUDA runtime or driver error                 */
+#define WISE_ERR_WORKSPACE (-6)/* workspace missing or too small               */
+
+/* Device status bits (wise_device_status). */
+#define WISE_STATUS_TIMEOUT 0x1u        /* a bounded pipeline wait expired        */
+#define WISE_STATUS_BAD_SCHEDULE 0x2u   /* schedule entry out of range / unsorted */
+
+#define WISE_BLOCK 32
+
+typedef struct wise_shape {
+  int32_t batch;
+  int32_t heads;
+  int32_t seqlen;
+  int32_t head_dim;
+  float scale; /* softmax temperature; <= 0 selects 1/sqrt(head_dim) (WISE paper section 3) */
+} wise_shape_t;
+
+/*
+ * Dense causal attention of one exploration step, optionally with block mass.
+ *
+ * Defines (WISE paper section 3, recurrent attention equation):
+ *   A = softmax(Q K^T * scale + M),  O = A V,  M_ij = -inf for j > i.
+ * and, when `mass` is non-NULL, the block mass of section 5.1:
+ *   mass[bh][q][b] = (1/32) sum_{i in block q} sum_{j in block b} A_ij,  b <= q.
+ *
+ * q, k, v : bf16 [B, H, n, d] inputs.
+ * o       : bf16 [B, H, n, d] output.
+ * lse     : fp32 [B, H, n] output, natural-log row normaliser
+ *           lse_i = log sum_{j<=i} exp(s_ij * scale); may be NULL unless
+ *           mass is requested (the mass pass reads it back).
+ * mass    : fp32 [B, H, nq, nq] output or NULL.  Only entries b <= q are
+ *           written; entries b > q are left untouched.
+ * Errors  : WISE_ERR_ARG (q/k/v/o NULL, mass without lse), WISE_ERR_SHAPE,
+ *           WISE_ERR_ALIGN, WISE_ERR_CUDA.
+ */
+int wise_full_attn_mass(const void* q, const void* k, const void* v, void* o, float* lse,
+                        float* mass, wise_shape_t shape, void* stream);
+
+/*
+ * Per-step cumulative-eta block support, OR-ed into the working set.
+ *
+ * Defines (WISE paper section 3 "attention support", section 6.1, and the
+ * temporal union of appendix B "WISE configuration"): for every (bh, q) the
+ * admissible blocks b <= q are ranked by mass[bh][q][b], descending, ties to
+ * the lower block index; the support is the shortest prefix whose cumulative
+ * mass is >= eta.  If eta >= 1, or no prefix reaches eta, every admissible
+ * block is kept.  Cumulative sums are taken in fp32.
+ *
+ * mass       : fp32 [B, H, nq, nq] (entries b > q are not read).
+ * union_bits : uint32 [B, H, nq, W], W = ceil(nq / 32), in/out.  Bit (b % 32)
+ *              of word b / 32 of row (bh, q) is set for every selected block
+ *              (bit-or accumulate).  The caller zeroes it before the first
+ *              window step.
+ * step_bits  : uint32 [B, H, nq, W] output of this step's support alone, or NULL.
+ * eta        : in (0, 1] ... values > 1 behave like 1.
+ * Errors     : WISE_ERR_ARG (NULL mass/union_bits, eta <= 0 or NaN), WISE_ERR_SHAPE,
+ *              WISE_ERR_CUDA.
+ */
+int wise_select_union(const float* mass, uint32_t* union_bits, uint32_t* step_bits, float eta,
+                      wise_shape_t shape, void* stream);
+
+/* Workspace bytes wise_build_schedule needs for this shape (device memory). */
+size_t wise_schedule_workspace_bytes(wise_shape_t shape);
+
+/* Largest possible schedule size: BH * nq * (nq + 1) / 2 entries. */
+int64_t wise_schedule_max_nnz(wise_shape_t shape);
+
+/*
+ * Compact the working set into the GPU-resident CSR schedule (WISE paper,
+ * appendix B "Sparse-kernel implementation": row offsets plus active block
+ * indices per recurrent block, head and query block).
+ *
+ * union_bits  : uint32 [B, H, nq, W] as produced by wise_select_union.  Bits
+ *               for blocks b > q are ignored.
+ * row_offsets : int32 [B*H*nq + 1] output; row r = bh * nq + q spans
+ *               col_idx[row_offsets[r] .. row_offsets[r+1]).
+ * col_idx     : int32 [col_capacity] output, key-block indices ascending per row.
+ * nnz_out     : HOST int64 pointer or NULL.  If non-NULL the call synchronises
+ *               `stream`, stores the entry count and returns WISE_ERR_CAPACITY
+ *               if it exceeds col_capacity (col_idx then holds the first
+ *               col_capacity entries).  If NULL, col_capacity must be at least
+ *               wise_schedule_max_nnz(shape).
+ * workspace   : device scratch of at least wise_schedule_workspace_bytes(shape).
+ * Errors      : WISE_ERR_ARG, WISE_ERR_SHAPE, WISE_ERR_WORKSPACE, WISE_ERR_CAPACITY,
+ *               WISE_ERR_CUDA.
+ */
+int wise_build_schedule(const uint32_t* union_bits, int32_t* row_offsets, int32_t* col_idx,
+                        int64_t col_capacity, int64_t* nnz_out, void* workspace,
+                        size_t workspace_bytes, wise_shape_t shape, void* stream);
+
+/*
+ * Late-step block-sparse causal attention over a CSR schedule.
+ *
+ * Defines (WISE paper section 5.2, reuse mask R, and section 7.4): the dense
+ * attention of wise_full_attn_mass restricted to keys j with j <= i and
+ * block(j) in the schedule row of block(i); absent blocks are skipped, not
+ * masked.  Q, K, V are this step's fresh values.
+ *
+ * row_offsets, col_idx : the schedule (see wise_build_schedule); each row's
+ *               indices must be ascending and <= its query block.  Entries
+ *               outside [0, col_count) or violating that order are skipped and
+ *               flag WISE_STATUS_BAD_SCHEDULE; they never cause an out-of-range
+ *               access.
+ * col_count   : number of valid entries in col_idx (row_offsets[B*H*nq]).
+ * lse         : fp32 [B, H, n] output or NULL.
+ * A row whose schedule row is empty gets O = 0 and lse = -inf.
+ * Errors      : WISE_ERR_ARG, WISE_ERR_SHAPE, WISE_ERR_ALIGN, WISE_ERR_CUDA.
+ */
+int wise_sparse_attn(const void* q, const void* k, const void* v, void* o,
+                     const int32_t* row_offsets, const int32_t* col_idx, int64_t col_count,
+                     float* lse, wise_shape_t shape, void* stream);
+
+/*
+ * Read (and optionally clear) the device status word of the current device.
+ * Synchronises the device.  *status_out receives WISE_STATUS_* bits.
+ */
+int wise_device_status(uint32_t* status_out, int clear);
+
+/* Message of the last error returned on this thread ("" if none). */
+const char* wise_last_error(void);
+
+/* Library version string. */
+const char* wise_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WISE_H_ */

@@ -1,0 +1,294 @@
+// api.cu -- the C ABI of libwise (include/wise.h): argument validation,
+// TMA descriptor construction and kernel launches.  No entry point allocates
+// device memory; only wise_build_schedule with nnz_out and wise_device_status
+// synchronise.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "wise.h"
+#include "wise_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int ok() {
+  g_last_error.clear();
+  return WISE_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(WISE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+}  // namespace
+
+namespace wise {
+__device__ unsigned int g_status_word = 0u;
+}
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool init = false;
+  int sms = 0;
+  unsigned int* status = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(WISE_ERR_CUDA, "device index %d unsupported", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.init) {
+    e = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, wise::g_status_word);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+    di.status = static_cast<unsigned int*>(p);
+    di.init = true;
+  }
+  *out = &di;
+  return WISE_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [BH, n, d] bf16 viewed as a 3-D tensor (d fastest); box = 64 columns x box_rows rows,
+// 128-byte swizzle, zero fill outside the tensor.
+int make_tmap(CUtensorMap* map, const void* base, int d, int n, int BH, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(WISE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * (cuuint64_t)n};
+  cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(WISE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return WISE_OK;
+}
+
+int check_shape(const wise_shape_t& s) {
+  if (s.batch < 1 || s.heads < 1)
+    return fail(WISE_ERR_SHAPE, "batch (%d) and heads (%d) must be >= 1", s.batch, s.heads);
+  if (s.seqlen < 32 || s.seqlen % 32 != 0 || s.seqlen > 16384)
+    return fail(WISE_ERR_SHAPE, "seqlen %d must be a multiple of 32 in [32, 16384]", s.seqlen);
+  if (s.head_dim != 64 && s.head_dim != 96 && s.head_dim != 128)
+    return fail(WISE_ERR_SHAPE, "head_dim %d unsupported (64, 96 or 128)", s.head_dim);
+  const long long bh = (long long)s.batch * s.heads;
+  if (bh > (1ll << 24)) return fail(WISE_ERR_SHAPE, "batch*heads %lld too large", bh);
+  if (!(std::isfinite(s.scale))) return fail(WISE_ERR_ARG, "scale must be finite");
+  return WISE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+float softmax_scale(const wise_shape_t& s) {
+  return s.scale > 0.f ? s.scale : 1.0f / std::sqrt((float)s.head_dim);
+}
+
+int launch_attn(int mode, const void* q, const void* k, const void* v, void* o,
+                const wise::AttnParams& p0, const wise_shape_t& s, void* stream) {
+  DeviceInfo* di = nullptr;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  const int BH = s.batch * s.heads;
+  CUtensorMap tq, tk, tv, to;
+  if ((rc = make_tmap(&tq, q, s.head_dim, s.seqlen, BH, 128))) return rc;
+  if ((rc = make_tmap(&tk, k, s.head_dim, s.seqlen, BH, 32))) return rc;
+  if (mode != wise::kModeMass) {
+    if ((rc = make_tmap(&tv, v, s.head_dim, s.seqlen, BH, 32))) return rc;
+    if ((rc = make_tmap(&to, o, s.head_dim, s.seqlen, BH, 128))) return rc;
+  } else {
+    tv = tk;
+    to = tq;
+  }
+  wise::AttnParams p = p0;
+  p.BH = BH;
+  p.n = s.seqlen;
+  p.nq = s.seqlen / 32;
+  p.num_tiles = BH * ((p.nq + 3) / 4);
+  p.scale_log2 = softmax_scale(s) * 1.4426950408889634f;
+  p.status = di->status;
+  const int grid = p.num_tiles < di->sms ? p.num_tiles : di->sms;
+  cudaError_t e = wise::launch_attention(mode, s.head_dim, tq, tk, tv, to, p, grid,
+                                         static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  return WISE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int wise_full_attn_mass(const void* q, const void* k, const void* v, void* o, float* lse,
+                        float* mass, wise_shape_t shape, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!q || !k || !v || !o) return fail(WISE_ERR_ARG, "q, k, v and o must be non-NULL");
+  if (mass && !lse) return fail(WISE_ERR_ARG, "mass requires an lse buffer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(WISE_ERR_ALIGN, "q, k, v, o must be 16-byte aligned");
+  if ((lse && !aligned16(lse)) || (mass && !aligned16(mass)))
+    return fail(WISE_ERR_ALIGN, "lse and mass must be 16-byte aligned");
+  wise::AttnParams p{};
+  p.lse = lse;
+  rc = launch_attn(wise::kModeDense, q, k, v, o, p, shape, stream);
+  if (rc) return rc;
+  if (mass) {
+    wise::AttnParams pm{};
+    pm.lse_in = lse;
+    pm.mass = mass;
+    rc = launch_attn(wise::kModeMass, q, k, v, o, pm, shape, stream);
+    if (rc) return rc;
+  }
+  return ok();
+}
+
+int wise_select_union(const float* mass, uint32_t* union_bits, uint32_t* step_bits, float eta,
+                      wise_shape_t shape, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!mass || !union_bits) return fail(WISE_ERR_ARG, "mass and union_bits must be non-NULL");
+  if (!(eta > 0.f)) return fail(WISE_ERR_ARG, "eta must be > 0 (got %g)", (double)eta);
+  const int nq = shape.seqlen / 32;
+  cudaError_t e = wise::launch_select_union(mass, union_bits, step_bits, eta,
+                                            shape.batch * shape.heads, nq,
+                                            static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "select_union launch");
+  return ok();
+}
+
+size_t wise_schedule_workspace_bytes(wise_shape_t shape) {
+  if (check_shape(shape)) return 0;
+  const long long rows = (long long)shape.batch * shape.heads * (shape.seqlen / 32);
+  return wise::schedule_workspace_bytes(rows);
+}
+
+int64_t wise_schedule_max_nnz(wise_shape_t shape) {
+  if (check_shape(shape)) return -1;
+  const long long nq = shape.seqlen / 32;
+  return (long long)shape.batch * shape.heads * nq * (nq + 1) / 2;
+}
+
+int wise_build_schedule(const uint32_t* union_bits, int32_t* row_offsets, int32_t* col_idx,
+                        int64_t col_capacity, int64_t* nnz_out, void* workspace,
+                        size_t workspace_bytes, wise_shape_t shape, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!union_bits || !row_offsets || !col_idx)
+    return fail(WISE_ERR_ARG, "union_bits, row_offsets and col_idx must be non-NULL");
+  if (col_capacity < 0) return fail(WISE_ERR_ARG, "col_capacity must be >= 0");
+  const long long nq = shape.seqlen / 32;
+  const long long rows = (long long)shape.batch * shape.heads * nq;
+  const long long max_nnz = rows * (nq + 1) / 2;
+  if (max_nnz > 0x7fffffffll) return fail(WISE_ERR_SHAPE, "schedule may exceed 2^31 entries");
+  const size_t need = wise::schedule_workspace_bytes(rows);
+  if (!workspace || workspace_bytes < need)
+    return fail(WISE_ERR_WORKSPACE, "workspace of %zu bytes required", need);
+  if (!nnz_out && col_capacity < max_nnz)
+    return fail(WISE_ERR_CAPACITY,
+                "col_capacity %lld < worst case %lld; pass nnz_out to check the exact size",
+                (long long)col_capacity, max_nnz);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = wise::launch_build_schedule(union_bits, row_offsets, col_idx, col_capacity,
+                                              workspace, rows, (int)nq, st);
+  if (e != cudaSuccess) return cuda_fail(e, "build_schedule launch");
+  if (nnz_out) {
+    int32_t nnz = 0;
+    e = cudaMemcpyAsync(&nnz, row_offsets + rows, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "reading nnz");
+    *nnz_out = nnz;
+    if (nnz > col_capacity)
+      return fail(WISE_ERR_CAPACITY, "schedule has %d entries, capacity %lld", nnz,
+                  (long long)col_capacity);
+  }
+  return ok();
+}
+
+int wise_sparse_attn(const void* q, const void* k, const void* v, void* o,
+                     const int32_t* row_offsets, const int32_t* col_idx, int64_t col_count,
+                     float* lse, wise_shape_t shape, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !row_offsets || (!col_idx && col_count > 0))
+    return fail(WISE_ERR_ARG, "q, k, v, o, row_offsets, col_idx must be non-NULL");
+  if (col_count < 0) return fail(WISE_ERR_ARG, "col_count must be >= 0");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(WISE_ERR_ALIGN, "q, k, v, o must be 16-byte aligned");
+  wise::AttnParams p{};
+  p.lse = lse;
+  p.row_offsets = row_offsets;
+  p.col_idx = col_idx;
+  p.col_count = col_count;
+  rc = launch_attn(wise::kModeSparse, q, k, v, o, p, shape, stream);
+  if (rc) return rc;
+  return ok();
+}
+
+int wise_device_status(uint32_t* status_out, int clear) {
+  if (!status_out) return fail(WISE_ERR_ARG, "status_out must be non-NULL");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  unsigned int v = 0;
+  e = cudaMemcpyFromSymbol(&v, wise::g_status_word, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "reading status");
+  *status_out = v;
+  if (clear) {
+    const unsigned int z = 0;
+    e = cudaMemcpyToSymbol(wise::g_status_word, &z, sizeof(z));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing status");
+  }
+  return ok();
+}
+
+const char* wise_last_error(void) { return g_last_error.c_str(); }
+
+const char* wise_version(void) { return "wise-b200 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,40 @@
+// wise_internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace wise {
+
+enum { kModeDense = 0, kModeSparse = 1, kModeMass = 2 };
+
+struct AttnParams {
+  int BH;               // batch * heads
+  int n;                // sequence length
+  int nq;               // n / 32
+  int num_tiles;        // BH * ceil(nq / 4)
+  float scale_log2;     // softmax scale * log2(e)
+  float* lse;           // [BH, n] output (dense / sparse), nullable
+  const float* lse_in;  // [BH, n] input (mass mode)
+  float* mass;          // [BH, nq, nq] output (mass mode)
+  const int32_t* row_offsets;  // sparse mode
+  const int32_t* col_idx;      // sparse mode
+  long long col_count;         // sparse mode: valid entries of col_idx
+  unsigned int* status;        // device status word
+};
+
+cudaError_t launch_attention(int mode, int d, const CUtensorMap& tq, const CUtensorMap& tk,
+                             const CUtensorMap& tv, const CUtensorMap& to, const AttnParams& p,
+                             int grid, cudaStream_t stream);
+int attention_smem_bytes(int mode, int d);
+
+cudaError_t launch_select_union(const float* mass, uint32_t* union_bits, uint32_t* step_bits,
+                                float eta, int BH, int nq, cudaStream_t stream);
+
+size_t schedule_workspace_bytes(long long rows);
+cudaError_t launch_build_schedule(const uint32_t* union_bits, int32_t* row_offsets,
+                                  int32_t* col_idx, long long capacity, void* workspace,
+                                  long long rows, int nq, cudaStream_t stream);
+
+}  // namespace wise

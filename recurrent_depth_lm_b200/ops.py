@@ -1,0 +1,141 @@
+"""torch-tensor front end of the C ABI (argument marshalling only).
+
+Tensors are device tensors owned by the caller (or allocated here with torch
+when an output is not supplied); the library itself never allocates.  Every
+function launches on the current torch CUDA stream unless `stream` is given.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+
+import torch
+
+from . import _lib
+from ._lib import WiseShape, check, lib
+
+BLOCK = 32
+
+
+def shape_of(q: torch.Tensor, scale: float | None = None) -> WiseShape:
+    if q.dim() != 4:
+        raise ValueError("expected [batch, heads, seqlen, head_dim]")
+    b, h, n, d = q.shape
+    return WiseShape(b, h, n, d, float(scale) if scale else 0.0)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _check_qkv(*ts: torch.Tensor) -> None:
+    ref = ts[0]
+    for t in ts:
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("q/k/v/o must be contiguous bf16 CUDA tensors")
+        if t.shape != ref.shape:
+            raise ValueError("q/k/v/o shapes differ")
+
+
+def words_per_row(nq: int) -> int:
+    return (nq + 31) // 32
+
+
+def full_attn_mass(q, k, v, *, with_mass: bool = False, o=None, lse=None, mass=None,
+                   scale=None, stream=None):
+    """Dense causal attention (+ block mass).  Returns (o, lse, mass)."""
+    b, h, n, d = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    _check_qkv(q, k, v, o)
+    if with_mass and mass is None:
+        mass = torch.empty(b, h, n // BLOCK, n // BLOCK, dtype=torch.float32, device=q.device)
+    if (with_mass or mass is not None) and lse is None:
+        lse = torch.empty(b, h, n, dtype=torch.float32, device=q.device)
+    rc = lib.wise_full_attn_mass(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(mass),
+                                 shape_of(q, scale), _stream(stream))
+    check(rc, "wise_full_attn_mass")
+    return o, lse, mass
+
+
+def select_union(mass, union_bits, eta: float, *, step_bits=None, head_dim: int = 128,
+                 scale=None, stream=None):
+    """OR the cumulative-eta support of `mass` into `union_bits` (in place)."""
+    b, h, nq, _ = mass.shape
+    shp = WiseShape(b, h, nq * BLOCK, head_dim, float(scale) if scale else 0.0)
+    if mass.dtype != torch.float32 or union_bits.dtype != torch.int32:
+        raise ValueError("mass must be float32 and union_bits int32 (uint32 bit patterns)")
+    rc = lib.wise_select_union(_ptr(mass), _ptr(union_bits), _ptr(step_bits), float(eta), shp,
+                               _stream(stream))
+    check(rc, "wise_select_union")
+    return union_bits
+
+
+def new_bitmask(b: int, h: int, nq: int, device) -> torch.Tensor:
+    return torch.zeros(b, h, nq, words_per_row(nq), dtype=torch.int32, device=device)
+
+
+def schedule_workspace(b: int, h: int, n: int, head_dim: int, device) -> torch.Tensor:
+    nbytes = lib.wise_schedule_workspace_bytes(WiseShape(b, h, n, head_dim, 0.0))
+    return torch.empty(max(1, nbytes), dtype=torch.uint8, device=device)
+
+
+def schedule_max_nnz(b: int, h: int, n: int, head_dim: int = 128) -> int:
+    return int(lib.wise_schedule_max_nnz(WiseShape(b, h, n, head_dim, 0.0)))
+
+
+def build_schedule(union_bits, *, head_dim: int = 128, row_offsets=None, col_idx=None,
+                   workspace=None, exact_nnz: bool = True, stream=None):
+    """CSR schedule of the working set.  Returns (row_offsets, col_idx, nnz or None)."""
+    b, h, nq, _ = union_bits.shape
+    n = nq * BLOCK
+    dev = union_bits.device
+    if row_offsets is None:
+        row_offsets = torch.empty(b * h * nq + 1, dtype=torch.int32, device=dev)
+    if col_idx is None:
+        col_idx = torch.empty(schedule_max_nnz(b, h, n, head_dim), dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = schedule_workspace(b, h, n, head_dim, dev)
+    nnz = ctypes.c_int64(-1)
+    rc = lib.wise_build_schedule(_ptr(union_bits), _ptr(row_offsets), _ptr(col_idx),
+                                 col_idx.numel(), ctypes.byref(nnz) if exact_nnz else None,
+                                 _ptr(workspace), workspace.numel(),
+                                 WiseShape(b, h, n, head_dim, 0.0), _stream(stream))
+    check(rc, "wise_build_schedule")
+    return row_offsets, col_idx, (int(nnz.value) if exact_nnz else None)
+
+
+def sparse_attn(q, k, v, row_offsets, col_idx, col_count: int | None = None, *, o=None,
+                lse=None, scale=None, stream=None):
+    """Block-sparse causal attention over a CSR schedule.  Returns (o, lse)."""
+    if o is None:
+        o = torch.empty_like(q)
+    _check_qkv(q, k, v, o)
+    if col_count is None:
+        col_count = col_idx.numel()
+    rc = lib.wise_sparse_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(row_offsets),
+                              _ptr(col_idx), int(col_count), _ptr(lse), shape_of(q, scale),
+                              _stream(stream))
+    check(rc, "wise_sparse_attn")
+    return o, lse
+
+
+def device_status(clear: bool = True) -> int:
+    st = ctypes.c_uint32(0)
+    check(lib.wise_device_status(ctypes.byref(st), 1 if clear else 0), "wise_device_status")
+    return int(st.value)
+
+
+def causal_flops(n: int, d: int, bh: int) -> float:
+    """Useful FLOPs of dense causal attention: 4*d per admissible (i, j) pair."""
+    return 4.0 * d * bh * n * (n + 1) / 2
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)

@@ -1,0 +1,87 @@
+"""WISE trajectory driver for one attention layer (the user-facing API).
+
+Wan & Chen, "Attention Routing Stabilizes Early: Working-Set Inference for
+Recurrent-Depth Language Models", section 5 and appendix B: steps
+t <= t_d run unrestricted (dense) causal attention; steps t_d-3 .. t_d also
+select each query block's cumulative-eta key-block support and union it;
+after step t_d the union is compacted once into a CSR schedule; every later
+step runs block-sparse attention over that schedule with fresh Q, K, V.
+
+All buffers are allocated once here with torch; the library calls only
+enqueue kernels on the current stream (no host synchronisation inside a
+trajectory).
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import ops
+
+
+class WiseTrajectory:
+    def __init__(self, batch: int, heads: int, seqlen: int, head_dim: int, *, t_d: int = 12,
+                 window=(9, 12), eta: float = 0.95, scale: float | None = None,
+                 device="cuda", keep_step_bits: bool = False):
+        if seqlen % ops.BLOCK:
+            raise ValueError("seqlen must be a multiple of 32")
+        self.b, self.h, self.n, self.d = batch, heads, seqlen, head_dim
+        self.nq = seqlen // ops.BLOCK
+        self.t_d, self.window, self.eta = t_d, tuple(window), float(eta)
+        self.scale = scale
+        dev = torch.device(device)
+        self.lse = torch.empty(batch, heads, seqlen, dtype=torch.float32, device=dev)
+        self.mass = torch.empty(batch, heads, self.nq, self.nq, dtype=torch.float32, device=dev)
+        self.union = ops.new_bitmask(batch, heads, self.nq, dev)
+        self.step_bits = {}
+        self.keep_step_bits = keep_step_bits
+        self.row_offsets = torch.empty(batch * heads * self.nq + 1, dtype=torch.int32, device=dev)
+        self.col_idx = torch.empty(ops.schedule_max_nnz(batch, heads, seqlen, head_dim),
+                                   dtype=torch.int32, device=dev)
+        self.workspace = ops.schedule_workspace(batch, heads, seqlen, head_dim, dev)
+        self.scheduled = False
+
+    def reset(self) -> None:
+        self.union.zero_()
+        self.step_bits.clear()
+        self.scheduled = False
+
+    def in_window(self, t: int) -> bool:
+        return self.window[0] <= t <= self.window[1]
+
+    def step(self, t: int, q, k, v, o=None, lse=None, stream=None):
+        """Attention of recurrent step t (1-based).  Returns O."""
+        if t <= self.t_d:
+            if self.in_window(t):
+                o, _, _ = ops.full_attn_mass(q, k, v, o=o, lse=self.lse, mass=self.mass,
+                                             scale=self.scale, stream=stream)
+                sb = None
+                if self.keep_step_bits:
+                    sb = torch.empty_like(self.union)
+                    self.step_bits[t] = sb
+                ops.select_union(self.mass, self.union, self.eta, step_bits=sb,
+                                 head_dim=self.d, scale=self.scale, stream=stream)
+            else:
+                o, _, _ = ops.full_attn_mass(q, k, v, o=o, lse=lse, scale=self.scale,
+                                             stream=stream)
+            if t == self.t_d:
+                self.build_schedule(stream=stream)
+            return o
+        if not self.scheduled:
+            raise RuntimeError("late step before the schedule was built (t <= t_d never reached)")
+        o, _ = ops.sparse_attn(q, k, v, self.row_offsets, self.col_idx, self.col_idx.numel(),
+                               o=o, lse=lse, scale=self.scale, stream=stream)
+        return o
+
+    def build_schedule(self, stream=None) -> None:
+        ops.build_schedule(self.union, head_dim=self.d, row_offsets=self.row_offsets,
+                           col_idx=self.col_idx, workspace=self.workspace, exact_nnz=False,
+                           stream=stream)
+        self.scheduled = True
+
+    def nnz(self) -> int:
+        return int(self.row_offsets[-1].item())
+
+    def density(self) -> float:
+        """Fraction of admissible (causal) query-key blocks retained."""
+        return self.nnz() / (self.b * self.h * self.nq * (self.nq + 1) / 2)

@@ -1,0 +1,102 @@
+"""The C-ABI library loads, exports every declared symbol, and rejects bad
+arguments on the host (no GPU needed: validation happens before any launch)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[\w]+\s*\*?\s*(wise_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from recurrent_depth_lm_b200 import _lib
+    return _lib
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 9, names
+    raw = ctypes.CDLL(lib.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), n
+    assert set(names) == set(lib._SIGNATURES), "binding and header disagree"
+
+
+def test_version(lib):
+    assert "sm_100a" in lib.version()
+
+
+def shape(lib, b=1, h=2, n=256, d=64, s=0.0):
+    return lib.WiseShape(b, h, n, d, s)
+
+
+@pytest.mark.parametrize("b,h,n,d", [(0, 1, 256, 64), (1, 0, 256, 64), (1, 1, 100, 64),
+                                     (1, 1, 0, 64), (1, 1, 32768, 64), (1, 1, 256, 80),
+                                     (1, 1, 256, 256)])
+def test_bad_shapes_rejected(lib, b, h, n, d):
+    L = lib.lib
+    fake = 1 << 20
+    rc = L.wise_full_attn_mass(fake, fake, fake, fake, None, None, shape(lib, b, h, n, d), None)
+    assert rc == lib.WISE_ERR_SHAPE, lib.last_error()
+    rc = L.wise_sparse_attn(fake, fake, fake, fake, fake, fake, 1, None, shape(lib, b, h, n, d), None)
+    assert rc == lib.WISE_ERR_SHAPE
+    assert L.wise_schedule_max_nnz(shape(lib, b, h, n, d)) == -1
+
+
+def test_null_and_alignment_rejected(lib):
+    L = lib.lib
+    s = shape(lib)
+    assert L.wise_full_attn_mass(None, 16, 16, 16, None, None, s, None) == lib.WISE_ERR_ARG
+    assert L.wise_full_attn_mass(16, 16, 16, 16, None, 16, s, None) == lib.WISE_ERR_ARG  # mass w/o lse
+    assert L.wise_full_attn_mass(18, 16, 16, 16, None, None, s, None) == lib.WISE_ERR_ALIGN
+    assert L.wise_sparse_attn(16, 16, 16, 16, None, 16, 1, None, s, None) == lib.WISE_ERR_ARG
+    assert L.wise_sparse_attn(16, 16, 16, 16, 16, 16, -1, None, s, None) == lib.WISE_ERR_ARG
+    assert L.wise_sparse_attn(16, 16, 24, 16, 16, 16, 1, None, s, None) == lib.WISE_ERR_ALIGN
+    assert L.wise_select_union(None, 16, None, 0.95, s, None) == lib.WISE_ERR_ARG
+    assert L.wise_select_union(16, 16, None, 0.0, s, None) == lib.WISE_ERR_ARG
+    assert L.wise_select_union(16, 16, None, float("nan"), s, None) == lib.WISE_ERR_ARG
+    assert "eta" in lib.last_error()
+
+
+def test_schedule_sizes_and_checks(lib):
+    L = lib.lib
+    s = shape(lib, 1, 32, 4096, 128)
+    assert L.wise_schedule_max_nnz(s) == 32 * 128 * 129 // 2
+    ws = L.wise_schedule_workspace_bytes(s)
+    assert ws >= 4 * ((32 * 128 + 1023) // 1024)
+    # workspace missing / too small
+    rc = L.wise_build_schedule(16, 16, 16, 10 ** 9, None, None, 0, s, None)
+    assert rc == lib.WISE_ERR_WORKSPACE
+    # capacity below the worst case without nnz_out
+    rc = L.wise_build_schedule(16, 16, 16, 10, None, 16, ws, s, None)
+    assert rc == lib.WISE_ERR_CAPACITY
+    assert L.wise_build_schedule(None, 16, 16, 10, None, 16, ws, s, None) == lib.WISE_ERR_ARG
+
+
+def test_last_error_is_thread_local(lib):
+    import threading
+    L = lib.lib
+    L.wise_select_union(None, None, None, 0.5, shape(lib), None)
+    seen = {}
+
+    def other():
+        seen["msg"] = lib.last_error()
+
+    t = threading.Thread(target=other)
+    t.start()
+    t.join()
+    assert seen["msg"] == ""
+    assert lib.last_error() != ""

@@ -1,0 +1,262 @@
+"""GPU-vs-oracle parity of each C-ABI entry point on seeded random inputs.
+
+Sizes span several 128-row tiles, ragged tails (seqlen not a multiple of 128,
+a single 32-token block), every supported head_dim and batch*heads > 1.
+"""
+
+import numpy as np
+import pytest
+
+from oracle import wise_oracle as O
+from parity_utils import (LSE_TOL, MASS_TOL, bits_to_bool, check_csr, compare_o,
+                          compare_selection)
+from wise_inputs import bf16_bits_to_f64, f32_to_bf16_bits
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def ops():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from recurrent_depth_lm_b200 import ops as _ops
+    return _ops
+
+
+def rand_qkv_bits(b, h, n, d, seed, qscale=2.0):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((b, h, n, d), dtype=np.float32) * np.float32(qscale)
+    k = rng.standard_normal((b, h, n, d), dtype=np.float32)
+    v = rng.standard_normal((b, h, n, d), dtype=np.float32)
+    return [f32_to_bf16_bits(x) for x in (q, k, v)]
+
+
+def to_dev(bits):
+    return torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def dev_f32(t):
+    return t.float().cpu().numpy()
+
+
+SHAPES = [(1, 2, 256, 64), (1, 1, 32, 128), (2, 3, 160, 96), (1, 2, 544, 128), (1, 1, 1024, 96)]
+
+
+@pytest.mark.parametrize("b,h,n,d", SHAPES)
+def test_dense_attention_lse_and_mass(ops, b, h, n, d):
+    qb, kb, vb = rand_qkv_bits(b, h, n, d, seed=n + d)
+    q, k, v = to_dev(qb), to_dev(kb), to_dev(vb)
+    o, lse, mass = ops.full_attn_mass(q, k, v, with_mass=True)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    o, lse, mass = dev_f32(o), lse.cpu().numpy(), mass.cpu().numpy()
+    for bi in range(b):
+        for hi in range(h):
+            qf, kf, vf = (bf16_bits_to_f64(x[bi, hi]) for x in (qb, kb, vb))
+            o_ref, lse_ref = O.causal_attention(qf, kf, vf)
+            compare_o(o[bi, hi], o_ref, f"O[{bi},{hi}]")
+            assert np.abs(lse[bi, hi] - lse_ref).max() <= LSE_TOL
+            r_ref = O.block_mass(qf, kf)
+            m = np.tril(mass[bi, hi])
+            assert np.abs(m - r_ref).max() <= MASS_TOL
+
+
+def test_dense_without_lse(ops):
+    qb, kb, vb = rand_qkv_bits(1, 2, 96, 64, seed=5)
+    o, lse, mass = ops.full_attn_mass(to_dev(qb), to_dev(kb), to_dev(vb))
+    assert lse is None and mass is None
+    o = dev_f32(o)
+    for hi in range(2):
+        o_ref, _ = O.causal_attention(*(bf16_bits_to_f64(x[0, hi]) for x in (qb, kb, vb)))
+        compare_o(o[0, hi], o_ref)
+
+
+def random_support(nq, rng, p=0.4, diag=True, empty_rows=()):
+    s = np.tril(rng.random((nq, nq)) < p)
+    if diag:
+        s |= np.eye(nq, dtype=bool)
+    for r in empty_rows:
+        s[r] = False
+    return s
+
+
+def csr_device(supports):
+    """supports [BH][nq, nq] bool -> device row_offsets, col_idx (concatenated heads)."""
+    ros, cis, base = [0], [], 0
+    for s in supports:
+        ro, ci = O.csr_schedule(s)
+        ros.extend((ro[1:] + base).tolist())
+        cis.extend(ci.tolist())
+        base += len(ci)
+    ro = torch.tensor(ros, dtype=torch.int32, device="cuda")
+    ci = torch.tensor(cis if cis else [0], dtype=torch.int32, device="cuda")
+    return ro, ci, base
+
+
+@pytest.mark.parametrize("b,h,n,d", SHAPES)
+def test_sparse_attention_random_schedule(ops, b, h, n, d):
+    nq = n // 32
+    rng = np.random.default_rng(100 + n)
+    qb, kb, vb = rand_qkv_bits(b, h, n, d, seed=7 * n + d)
+    sups = [random_support(nq, rng, p=0.3) for _ in range(b * h)]
+    ro, ci, nnz = csr_device(sups)
+    lse = torch.empty(b, h, n, dtype=torch.float32, device="cuda")
+    o, _ = ops.sparse_attn(to_dev(qb), to_dev(kb), to_dev(vb), ro, ci, nnz, lse=lse)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    o, lse = dev_f32(o), lse.cpu().numpy()
+    for bi in range(b):
+        for hi in range(h):
+            qf, kf, vf = (bf16_bits_to_f64(x[bi, hi]) for x in (qb, kb, vb))
+            o_ref, lse_ref = O.masked_attention(qf, kf, vf, sups[bi * h + hi])
+            compare_o(o[bi, hi], o_ref, f"sparse O[{bi},{hi}]")
+            assert np.abs(lse[bi, hi] - lse_ref).max() <= LSE_TOL
+
+
+def test_sparse_all_blocks_equals_dense(ops):
+    b, h, n, d = 1, 2, 512, 128
+    nq = n // 32
+    qb, kb, vb = rand_qkv_bits(b, h, n, d, seed=11)
+    q, k, v = to_dev(qb), to_dev(kb), to_dev(vb)
+    full = np.tril(np.ones((nq, nq), dtype=bool))
+    ro, ci, nnz = csr_device([full] * (b * h))
+    o_s, _ = ops.sparse_attn(q, k, v, ro, ci, nnz)
+    o_d, _, _ = ops.full_attn_mass(q, k, v)
+    torch.cuda.synchronize()
+    # same kernel pipeline and the same block order: identical results
+    assert torch.equal(o_s, o_d)
+    o_ref, _ = O.causal_attention(*(bf16_bits_to_f64(x[0, 1]) for x in (qb, kb, vb)))
+    compare_o(dev_f32(o_s)[0, 1], o_ref)
+
+
+def test_sparse_diagonal_only_and_empty_rows(ops):
+    b, h, n, d = 1, 1, 256, 64
+    nq = n // 32
+    qb, kb, vb = rand_qkv_bits(b, h, n, d, seed=12)
+    sup = np.eye(nq, dtype=bool)
+    sup[3] = False      # an empty schedule row: O = 0, lse = -inf
+    sup[5, 0] = True
+    ro, ci, nnz = csr_device([sup])
+    lse = torch.empty(b, h, n, dtype=torch.float32, device="cuda")
+    o, _ = ops.sparse_attn(to_dev(qb), to_dev(kb), to_dev(vb), ro, ci, nnz, lse=lse)
+    torch.cuda.synchronize()
+    o, lse = dev_f32(o)[0, 0], lse.cpu().numpy()[0, 0]
+    qf, kf, vf = (bf16_bits_to_f64(x[0, 0]) for x in (qb, kb, vb))
+    rows = np.ones(n, dtype=bool)
+    rows[96:128] = False
+    o_ref, lse_ref = O.masked_attention(qf, kf, vf, sup)
+    compare_o(o[rows], o_ref[rows])
+    assert np.all(o[96:128] == 0.0) and np.all(np.isneginf(lse[96:128]))
+    assert np.abs(lse[rows] - lse_ref[rows]).max() <= LSE_TOL
+
+
+def test_sparse_bad_schedule_entries_are_skipped(ops):
+    """Entries above the diagonal or out of range are ignored and flagged, never read."""
+    b, h, n, d = 1, 1, 128, 64
+    nq = n // 32
+    qb, kb, vb = rand_qkv_bits(b, h, n, d, seed=13)
+    sup = np.tril(np.ones((nq, nq), dtype=bool))
+    ro, ci, nnz = csr_device([sup])
+    ci_h = ci.cpu().numpy()
+    ro_h = ro.cpu().numpy()
+    bad = ci_h.copy()
+    bad[ro_h[1]] = 3          # row 1 gets block 3 (> 1) instead of block 0
+    bad[ro_h[2]] = 1000       # row 2 gets an out-of-range block instead of block 0
+    ops.device_status(clear=True)
+    o, _ = ops.sparse_attn(to_dev(qb), to_dev(kb), to_dev(vb), ro,
+                           torch.tensor(bad, dtype=torch.int32, device="cuda"), nnz)
+    st = ops.device_status(clear=True)
+    assert st & 0x2
+    o = dev_f32(o)[0, 0]
+    eff = sup.copy()
+    eff[1, 0] = False
+    eff[2, 0] = False
+    o_ref, _ = O.masked_attention(*(bf16_bits_to_f64(x[0, 0]) for x in (qb, kb, vb)), eff)
+    compare_o(o, o_ref)
+
+
+@pytest.mark.parametrize("nq,bh", [(8, 2), (37, 3), (128, 2), (512, 1)])
+def test_select_union_matches_oracle(ops, nq, bh):
+    rng = np.random.default_rng(nq)
+    eta = 0.95
+    # masses from real softmax rows: peaky logits over admissible blocks
+    masses = np.zeros((bh, nq, nq))
+    for x in range(bh):
+        for q in range(nq):
+            lg = rng.standard_normal(q + 1) * 2.5
+            p = np.exp(lg - lg.max())
+            masses[x, q, : q + 1] = p / p.sum()
+    m32 = masses.astype(np.float32)
+    mass = torch.from_numpy(m32).reshape(1, bh, nq, nq).cuda()
+    union = ops.new_bitmask(1, bh, nq, "cuda")
+    step = torch.empty_like(union)
+    ops.select_union(mass, union, eta, step_bits=step)
+    # union accumulates: a second, different step ORs in
+    m2 = np.roll(m32, 1, axis=2) * np.tril(np.ones((nq, nq), np.float32))
+    m2 /= np.maximum(m2.sum(axis=2, keepdims=True), 1e-30)
+    step2 = torch.empty_like(union)
+    ops.select_union(torch.from_numpy(m2).reshape(1, bh, nq, nq).cuda(), union, eta,
+                     step_bits=step2)
+    torch.cuda.synchronize()
+    s1 = bits_to_bool(step.cpu().numpy()[0], nq)
+    s2 = bits_to_bool(step2.cpu().numpy()[0], nq)
+    u = bits_to_bool(union.cpu().numpy()[0], nq)
+    assert np.array_equal(u, s1 | s2)
+    for x in range(bh):
+        compare_selection(s1[x], m32[x].astype(np.float64), eta)
+        compare_selection(s2[x], m2[x].astype(np.float64), eta)
+        for q in range(nq):   # retained mass reaches eta
+            assert m32[x, q][s1[x, q]].astype(np.float64).sum() >= eta - 1e-6
+
+
+def test_select_eta_one_keeps_everything(ops):
+    nq, bh = 40, 2
+    m = np.tril(np.full((bh, nq, nq), 1.0 / nq, np.float32))
+    union = ops.new_bitmask(1, bh, nq, "cuda")
+    ops.select_union(torch.from_numpy(m).reshape(1, bh, nq, nq).cuda(), union, 1.0)
+    u = bits_to_bool(union.cpu().numpy()[0], nq)
+    assert np.array_equal(u, np.broadcast_to(np.tril(np.ones((nq, nq), bool)), u.shape))
+
+
+def test_select_golden_ties_and_exact_cut(ops):
+    """The hand-worked cases of tests/golden/eta_support_cases.json through the kernel."""
+    import json, os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "eta_support_cases.json")))
+    for c in g["cases"]:
+        r = np.array(c["r"], np.float32)
+        nq = len(r)
+        m = np.zeros((nq, nq), np.float32)
+        m[nq - 1, :] = r           # the case is the last query block's row
+        m[: nq - 1] = np.tril(np.ones((nq - 1, nq), np.float32)) / np.arange(1, nq)[:, None]
+        union = ops.new_bitmask(1, 1, nq, "cuda")
+        ops.select_union(torch.from_numpy(m).reshape(1, 1, nq, nq).cuda(), union, c["eta"])
+        u = bits_to_bool(union.cpu().numpy()[0, 0], nq)
+        assert np.nonzero(u[nq - 1])[0].tolist() == c["support"], c["why"]
+
+
+@pytest.mark.parametrize("nq,bh", [(1, 1), (8, 2), (45, 3), (512, 2)])
+def test_build_schedule_bit_exact(ops, nq, bh):
+    rng = np.random.default_rng(nq * 7 + bh)
+    bits = rng.integers(0, 2 ** 32, size=(1, bh, nq, (nq + 31) // 32), dtype=np.uint64)
+    dev_bits = torch.from_numpy(bits.astype(np.uint32).view(np.int32)).cuda()
+    ro, ci, nnz = ops.build_schedule(dev_bits, head_dim=64)
+    ro, ci = ro.cpu().numpy(), ci.cpu().numpy()
+    sup = np.tril(bits_to_bool(bits.astype(np.uint32)[0], nq))
+    assert nnz == int(sup.sum()) == ro[-1]
+    for x in range(bh):
+        r0, r1 = x * nq, (x + 1) * nq
+        check_csr(ro[r0:r1 + 1] - ro[r0], ci[ro[r0]:ro[r1]], sup[x])
+
+
+def test_build_schedule_capacity_error(ops):
+    from recurrent_depth_lm_b200._lib import WiseError
+    nq, bh = 16, 1
+    bits = torch.full((1, bh, nq, 1), -1, dtype=torch.int32, device="cuda")
+    small = torch.empty(10, dtype=torch.int32, device="cuda")
+    with pytest.raises(WiseError) as e:
+        ops.build_schedule(bits, col_idx=small, exact_nnz=True)
+    assert e.value.code == -4
+    with pytest.raises(WiseError):
+        ops.build_schedule(bits, col_idx=small, exact_nnz=False)
