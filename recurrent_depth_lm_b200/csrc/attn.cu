@@ -20,12 +20,10 @@
 // A slot's "owner mask" says which of the tile's 4 query blocks may see it;
 // rows of other query blocks get probability 0 for it.
 //
-// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM allocator +
-// single-thread MMA issuer, warps 2..5 = softmax / epilogue (one row each).
-//
 // Shared memory (128-byte swizzle, 1024-byte aligned panels of 64 columns):
-//   Q tile [128 x d], NS stages of K (and V) [128 keys x d], P [128 x 128] bf16.
-// Tensor memory: S double buffer (2 x 128 fp32 columns) + O (d columns).
+//   Q tile [128 x d], K and V stage rings [128 keys x d], P [128 x 128] bf16.
+// Tensor memory: S double buffer (2 x 128 fp32 columns) + one O accumulator
+// per softmax half (2 x 128 columns).
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -38,37 +36,46 @@ namespace wise {
 
 constexpr int kBM = 128;        // query rows per tile
 constexpr int kSlots = 4;       // key blocks per iteration
-constexpr int kThreads = 192;
-constexpr int kPanelRowBytes = 128;            // 64 bf16 per swizzled row
+constexpr int kThreads = 384;   // 12 warps
+constexpr int kPanelRowBytes = 128;                // 64 bf16 per swizzled row
 constexpr int kPanelBytes = kBM * kPanelRowBytes;  // one 128-row panel = 16 KB
 constexpr int kMaxWords = 16;   // schedule bitmask words per query block (nq <= 512)
+constexpr int kInfoRing = 8;    // iterations of slot info in flight
+constexpr int kSoftmaxThreads = 256;  // two halves of 4 warps
 
 template <int D, int MODE>
 struct Cfg {
   static constexpr int kPanels = (D + 63) / 64;
   static constexpr bool kAttn = MODE != kModeMass;
-  static constexpr int kStages = (D <= 64) ? 4 : (kAttn ? 2 : 4);
-  static constexpr int kTileBytes = kPanels * kPanelBytes;  // Q tile, K stage, V stage
+  static constexpr int kTileBytes = kPanels * kPanelBytes;  // Q tile, one K or V stage
+  // K ring (freed when QK finishes) and V ring (freed when PV finishes).
+  static constexpr int kKStages = kAttn ? (D <= 64 ? 4 : 3) : 4;
+  static constexpr int kVStages = kAttn ? (D <= 64 ? 4 : 2) : 0;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kTileBytes;
-  static constexpr int kOffV = kOffK + kStages * kTileBytes;
-  static constexpr int kOffP = kOffV + (kAttn ? kStages * kTileBytes : 0);
+  static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+  static constexpr int kOffP = kOffV + kVStages * kTileBytes;
   static constexpr int kOffInfo = kOffP + (kAttn ? 2 * kPanelBytes : 0);
-  static constexpr int kInfoInts = 16;
-  static constexpr int kOffMask = kOffInfo + kStages * kInfoInts * 4;
+  static constexpr int kInfoBytes = 64;
+  static constexpr int kOffMask = kOffInfo + kInfoRing * kInfoBytes;
   static constexpr int kOffBar = kOffMask + 4 * kMaxWords * 4;
-  // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full, o_done,
-  // o_staged, final
-  static constexpr int kNumBars = 2 + 2 * kStages + 4 + 4;
+  static constexpr int kVRing = kVStages > 0 ? kVStages : 1;  // barrier slots (mass mode: unused)
+  // q_full, q_empty, k_full[K], k_empty[K], v_full[V], v_empty[V], info_full[I], info_empty[I],
+  // s_full[2], s_free[2], p_full[2], o_done[2], merge, o_staged, final, spare
+  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVRing + 2 * kInfoRing + 12;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
   static constexpr uint32_t kTmemCols = kAttn ? 512 : 256;
-  static constexpr uint32_t kOCol = 256;
+  static constexpr uint32_t kOCol = 256;   // O of half h at kOCol + 128 * h
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kInfoRing >= kKStages + 1, "info slot reuse needs QK of its iteration done");
 };
 
 struct StageInfo {
   int nslots;
   int last;
+  int bh;
+  int pad;
   int kb[kSlots];
   int own[kSlots];
 };
@@ -85,6 +92,7 @@ struct DenseList {
     next = 0;
     end = min(qb0 + 3, nq - 1) + 1;
   }
+  __device__ bool empty() const { return next >= end; }
   __device__ bool pop(int& kb, int& own) {
     if (next >= end) return false;
     kb = next++;
@@ -108,12 +116,21 @@ struct MaskList {
     w = 0;
     cur = words > 0 ? (m[0] | m[kMaxWords] | m[2 * kMaxWords] | m[3 * kMaxWords]) : 0u;
   }
+  __device__ bool empty() const {
+    MaskList t = *this;
+    while (t.cur == 0) {
+      if (++t.w >= t.words) return true;
+      t.cur = t.mask[t.w] | t.mask[kMaxWords + t.w] | t.mask[2 * kMaxWords + t.w] |
+              t.mask[3 * kMaxWords + t.w];
+    }
+    return false;
+  }
   __device__ bool pop(int& kb, int& own) {
     while (cur == 0) {
       if (++w >= words) return false;
       cur = mask[w] | mask[kMaxWords + w] | mask[2 * kMaxWords + w] | mask[3 * kMaxWords + w];
     }
-    int bit = __ffs(cur) - 1;
+    const int bit = __ffs(cur) - 1;
     cur &= cur - 1;
     kb = w * 32 + bit;
     own = 0;
@@ -124,7 +141,8 @@ struct MaskList {
   }
 };
 
-// Build the 4 per-row bitmasks of a sparse tile (whole producer warp).
+// Build the 4 per-row bitmasks of a sparse tile (whole producer warp).  Entries
+// outside [0, q] or outside col_idx[0, col_count) are dropped and flagged.
 __device__ void build_tile_masks(uint32_t* mask, const AttnParams& p, int bh, int Qt, int lane) {
   const int words = (p.nq + 31) / 32;
   for (int x = lane; x < 4 * kMaxWords; x += 32) mask[x] = 0u;
@@ -154,9 +172,10 @@ __device__ void build_tile_masks(uint32_t* mask, const AttnParams& p, int bh, in
 
 // ---------------------------------------------------------------- helpers
 
-__device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
 #pragma unroll
-  for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i]));
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
 // Warp-uniform bounded wait: every lane polls, the warp agrees on the outcome.
@@ -175,6 +194,16 @@ __device__ __forceinline__ void decode_tile(int tile, int BH, int ntq, int& bh, 
 }
 
 // ---------------------------------------------------------------- the kernel
+//
+// Warp roles (384 threads): warp 0 = Q/K TMA producer and slot-list writer;
+// warp 1 = TMEM allocator + single-thread MMA issuer; warp 2 = V TMA producer;
+// warp 3 idle; warps 4..11 = softmax in two halves.  Half h (warps 4+4h ..
+// 7+4h) owns key slots 2h and 2h+1 of every iteration (S columns 64h..64h+63)
+// and keeps its own online-softmax state (m, l) and its own O accumulator in
+// TMEM; the two partial results of a row are merged once, in the epilogue:
+//   O = (2^(m_a-m) O_a + 2^(m_b-m) O_b) / (2^(m_a-m) l_a + 2^(m_b-m) l_b).
+// Warp w reads TMEM lane quarter w % 4 (rows 32*(w%4) .. +31), i.e. one query
+// block of the tile per warp.
 
 template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -182,6 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                 const AttnParams p) {
   using C = Cfg<D, MODE>;
+  constexpr int NK = C::kKStages;
+  constexpr int NV = C::kVRing;  // mass mode has no V ring; its barrier slots stay unused
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
 
@@ -197,15 +228,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar0 = smem_u32(smem + C::kOffBar);
   const uint32_t bar_q_full = bar0;
   const uint32_t bar_q_empty = bar0 + 8;
-  auto bar_kv_full = [&](int s) { return bar0 + 16 + 8 * s; };
-  auto bar_kv_empty = [&](int s) { return bar0 + 16 + 8 * C::kStages + 8 * s; };
-  const uint32_t barS = bar0 + 16 + 16 * C::kStages;
+  const uint32_t barK = bar0 + 16;
+  auto bar_k_full = [&](int s) { return barK + 8 * s; };
+  auto bar_k_empty = [&](int s) { return barK + 8 * NK + 8 * s; };
+  const uint32_t barV = barK + 16 * NK;
+  auto bar_v_full = [&](int s) { return barV + 8 * s; };
+  auto bar_v_empty = [&](int s) { return barV + 8 * NV + 8 * s; };
+  const uint32_t barI = barV + 16 * NV;
+  auto bar_i_full = [&](int s) { return barI + 8 * s; };
+  auto bar_i_empty = [&](int s) { return barI + 8 * kInfoRing + 8 * s; };
+  const uint32_t barS = barI + 16 * kInfoRing;
   auto bar_s_full = [&](int b) { return barS + 8 * b; };
   auto bar_s_free = [&](int b) { return barS + 16 + 8 * b; };
-  const uint32_t bar_p_full = barS + 32;
-  const uint32_t bar_o_done = barS + 40;
-  const uint32_t bar_o_staged = barS + 48;
-  const uint32_t bar_final = barS + 56;
+  auto bar_p_full = [&](int h) { return barS + 32 + 8 * h; };
+  auto bar_o_done = [&](int h) { return barS + 48 + 8 * h; };
+  const uint32_t bar_merge = barS + 64;
+  const uint32_t bar_o_staged = barS + 72;
+  const uint32_t bar_final = barS + 80;
   volatile int* abort_flag = (volatile int*)(smem + C::kOffMisc);
   uint32_t* tmem_slot = (uint32_t*)(smem + C::kOffMisc + 4);
 
@@ -215,19 +254,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     mbar_init(bar_q_full, 1);
     mbar_init(bar_q_empty, 1);
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(bar_kv_full(s), 1);
-      // mass mode: freed by the QK commit AND by every softmax thread once it has
-      // read the stage's slot info (128 + 1 arrivals); attention mode: by the PV commit.
-      mbar_init(bar_kv_empty(s), C::kAttn ? 1 : 129);
+    for (int s = 0; s < NK; ++s) {
+      mbar_init(bar_k_full(s), 1);
+      mbar_init(bar_k_empty(s), 1);
+    }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(bar_v_full(s), 1);
+      mbar_init(bar_v_empty(s), 1);
+    }
+    for (int s = 0; s < kInfoRing; ++s) {
+      mbar_init(bar_i_full(s), 1);
+      // read by the 256 softmax threads and, in attention modes, the V producer
+      mbar_init(bar_i_empty(s), kSoftmaxThreads + (C::kAttn ? 1 : 0));
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_s_full(b), 1);
-      mbar_init(bar_s_free(b), 128);
+      mbar_init(bar_s_free(b), kSoftmaxThreads);
+      mbar_init(bar_p_full(b), kSoftmaxThreads / 2);
+      mbar_init(bar_o_done(b), 1);
     }
-    mbar_init(bar_p_full, 128);
-    mbar_init(bar_o_done, 1);
-    mbar_init(bar_o_staged, 128);
+    mbar_init(bar_merge, kSoftmaxThreads);
+    mbar_init(bar_o_staged, kSoftmaxThreads);
     mbar_init(bar_final, 1);
     fence_mbar_init();
   }
@@ -241,14 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ======================================================= producer
+    // ======================================================= Q / K producer, slot lists
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
-      if (C::kAttn) {
-        tma_prefetch_desc(&tmV);
-        tma_prefetch_desc(&tmO);
-      }
     }
     uint32_t it = 0;
     int tl = 0;
@@ -256,10 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tl) {
       int bh, Qt;
       decode_tile(tile, p.BH, ntq, bh, Qt);
-      if (MODE == kModeSparse) {
-        // The previous tile's list has been fully issued (only lane 0 reads it).
-        build_tile_masks(tile_mask, p, bh, Qt, lane);
-      }
+      if (MODE == kModeSparse) build_tile_masks(tile_mask, p, bh, Qt, lane);
       if (lane == 0) {
         if (tl > 0 && !mbar_wait(bar_q_empty, (tl - 1) & 1, abort_flag, p.status)) ok = false;
         if (ok) {
@@ -275,53 +315,48 @@ __global__ void __launch_bounds__(kThreads, 1)
           dl.init(Qt, p.nq);
         bool first = true;
         while (ok) {
-          const int stage = it % C::kStages;
-          if (it >= (uint32_t)C::kStages &&
-              !mbar_wait(bar_kv_empty(stage), ((it / C::kStages) - 1) & 1, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          StageInfo& si = info[stage];
+          int kbv[kSlots], ownv[kSlots];
           int n = 0;
           int kb, own;
           while (n < kSlots && (MODE == kModeSparse ? ml.pop(kb, own) : dl.pop(kb, own))) {
-            si.kb[n] = kb;
-            si.own[n] = own;
+            kbv[n] = kb;
+            ownv[n] = own;
             ++n;
           }
-          if (n == 0 && first) {  // empty tile: one fully masked slot keeps the pipeline uniform
-            si.kb[0] = 0;
-            si.own[0] = 0;
+          if (n == 0) {
+            if (!first) break;  // unreachable: `last` was set on the previous group
+            kbv[0] = 0;         // empty tile: one fully masked slot keeps the pipeline uniform
+            ownv[0] = 0;
             n = 1;
           }
-          bool last;
-          if (n < kSlots) {
-            last = true;
-          } else {
-            // peek: is anything left?
-            if (MODE == kModeSparse) {
-              MaskList t = ml;
-              last = !t.pop(kb, own);
-            } else {
-              last = dl.next >= dl.end;
-            }
+          const bool last = (MODE == kModeSparse) ? ml.empty() : dl.empty();
+          const int is = it % kInfoRing;
+          if (it >= (uint32_t)kInfoRing &&
+              !mbar_wait(bar_i_empty(is), ((it / kInfoRing) - 1) & 1, abort_flag, p.status)) {
+            ok = false;
+            break;
           }
-          if (n == 0) break;  // cannot happen (handled above) but keeps the loop finite
+          StageInfo& si = info[is];
           si.nslots = n;
           si.last = last ? 1 : 0;
-          const uint32_t bytes = (uint32_t)n * 32 * kPanelRowBytes * C::kPanels * (C::kAttn ? 2 : 1);
-          mbar_arrive_expect_tx(bar_kv_full(stage), bytes);
-          const uint32_t kbase = sK + stage * C::kTileBytes;
-          const uint32_t vbase = sV + stage * C::kTileBytes;
-          for (int s = 0; s < n; ++s) {
-            for (int pn = 0; pn < C::kPanels; ++pn) {
-              tma_load_3d(kbase + pn * kPanelBytes + s * 32 * kPanelRowBytes, &tmK,
-                          bar_kv_full(stage), pn * 64, si.kb[s] * 32, bh);
-              if (C::kAttn)
-                tma_load_3d(vbase + pn * kPanelBytes + s * 32 * kPanelRowBytes, &tmV,
-                            bar_kv_full(stage), pn * 64, si.kb[s] * 32, bh);
-            }
+          si.bh = bh;
+          for (int s = 0; s < kSlots; ++s) {
+            si.kb[s] = s < n ? kbv[s] : 0;
+            si.own[s] = s < n ? ownv[s] : 0;
           }
+          mbar_arrive(bar_i_full(is));
+          const int ks = it % NK;
+          if (it >= (uint32_t)NK &&
+              !mbar_wait(bar_k_empty(ks), ((it / NK) - 1) & 1, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar_k_full(ks), (uint32_t)n * 32 * kPanelRowBytes * C::kPanels);
+          const uint32_t kbase = sK + ks * C::kTileBytes;
+          for (int s = 0; s < n; ++s)
+            for (int pn = 0; pn < C::kPanels; ++pn)
+              tma_load_3d(kbase + pn * kPanelBytes + s * 32 * kPanelRowBytes, &tmK, bar_k_full(ks),
+                          pn * 64, kbv[s] * 32, bh);
           ++it;
           first = false;
           if (last) break;
@@ -330,14 +365,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       it = __shfl_sync(0xffffffffu, it, 0);
     }
-    // Drain: let the last issued loads land before the CTA can exit.
-    if (lane == 0) {
-      const uint32_t from = it > (uint32_t)C::kStages ? it - C::kStages : 0u;
+    if (lane == 0) {  // let the last K loads land before the CTA can exit
+      const uint32_t from = it > (uint32_t)NK ? it - NK : 0u;
       for (uint32_t j = from; j < it; ++j) {
         volatile int dummy = 0;
-        mbar_wait(bar_kv_full(j % C::kStages), (j / C::kStages) & 1, &dummy, p.status);
+        mbar_wait(bar_k_full(j % NK), (j / NK) & 1, &dummy, p.status);
       }
     }
+  } else if (warp == 2) {
+    // ======================================================= V producer (attention modes)
+    if (C::kAttn && lane == 0) {
+      tma_prefetch_desc(&tmV);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        while (true) {
+          const int is = it % kInfoRing;
+          if (!mbar_wait(bar_i_full(is), (it / kInfoRing) & 1, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          const int n = info[is].nslots;
+          const int last = info[is].last;
+          const int bh = info[is].bh;
+          int kbv[kSlots];
+#pragma unroll
+          for (int s = 0; s < kSlots; ++s) kbv[s] = info[is].kb[s];
+          mbar_arrive(bar_i_empty(is));
+          const int vs = it % NV;
+          if (it >= (uint32_t)NV &&
+              !mbar_wait(bar_v_empty(vs), ((it / NV) - 1) & 1, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar_v_full(vs), (uint32_t)n * 32 * kPanelRowBytes * C::kPanels);
+          const uint32_t vbase = sV + vs * C::kTileBytes;
+          for (int s = 0; s < n; ++s)
+            for (int pn = 0; pn < C::kPanels; ++pn)
+              tma_load_3d(vbase + pn * kPanelBytes + s * 32 * kPanelRowBytes, &tmV, bar_v_full(vs),
+                          pn * 64, kbv[s] * 32, bh);
+          ++it;
+          if (last) break;
+        }
+      }
+      const uint32_t from = it > (uint32_t)NV ? it - NV : 0u;
+      for (uint32_t j = from; j < it; ++j) {
+        volatile int dummy = 0;
+        mbar_wait(bar_v_full(j % NV), (j / NV) & 1, &dummy, p.status);
+      }
+    }
+    __syncwarp();
   } else if (warp == 1) {
     // ======================================================= MMA issuer
     if (lane == 0) {
@@ -346,18 +423,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       int tl = 0;
       bool ok = true;
       bool issued = false;
-      // Issues S_j = Q K_j^T; returns the stage's slot count and last flag, read
-      // before the stage can be released.
+      // S_j = Q K_j^T into S buffer j&1; returns the iteration's slot count and last flag.
       auto issue_qk = [&](uint32_t j, int& ns, int& last) -> bool {
-        const int stage = j % C::kStages;
-        if (!mbar_wait(bar_kv_full(stage), (j / C::kStages) & 1, abort_flag, p.status)) return false;
-        if (j >= 2 && !mbar_wait(bar_s_free(j & 1), ((j >> 1) - 1) & 1, abort_flag, p.status)) return false;
+        const int ks = j % NK;
+        if (!mbar_wait(bar_k_full(ks), (j / NK) & 1, abort_flag, p.status)) return false;
+        if (j >= 2 && !mbar_wait(bar_s_free(j & 1), ((j >> 1) - 1) & 1, abort_flag, p.status))
+          return false;
         tc_fence_after();
-        ns = info[stage].nslots;
-        last = info[stage].last;
+        ns = info[j % kInfoRing].nslots;
+        last = info[j % kInfoRing].last;
         const uint32_t idesc = idesc_bf16_f32(128, 32 * ns, 0, 0);
         const uint32_t d_tmem = tmem_base + (j & 1) * 128;
-        const uint32_t kbase = sK + stage * C::kTileBytes;
+        const uint32_t kbase = sK + ks * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
@@ -365,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       smem_desc_sw128(kbase + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar_s_full(j & 1));
-        if (!C::kAttn) mma_commit(bar_kv_empty(stage));
+        mma_commit(bar_k_empty(ks));
         issued = true;
         return true;
       };
@@ -375,33 +452,46 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t g0 = it;
+        bool started[2] = {false, false};  // has half h's O been written in this tile
         int ns = 0, last = 1;
         if (!issue_qk(it, ns, last)) {
           ok = false;
           break;
         }
         while (true) {
-          const int stage = it % C::kStages;
           int ns_next = 0, last_next = 1;
           if (!last && !issue_qk(it + 1, ns_next, last_next)) {
             ok = false;
             break;
           }
           if (C::kAttn) {
-            if (!mbar_wait(bar_p_full, it & 1, abort_flag, p.status)) {
+            const int vs = it % NV;
+            if (!mbar_wait(bar_v_full(vs), (it / NV) & 1, abort_flag, p.status)) {
               ok = false;
               break;
             }
-            tc_fence_after();
-            const uint32_t vbase = sV + stage * C::kTileBytes;
-            for (int kk = 0; kk < 2 * ns; ++kk) {
-              const uint64_t a = smem_desc_sw128(sP + (kk >> 2) * kPanelBytes + (kk & 3) * 32, 16, 1024);
-              const uint64_t b = smem_desc_sw128(vbase + kk * 16 * kPanelRowBytes, kPanelBytes, 1024);
-              mma_bf16_ss(tmem_base + C::kOCol, a, b, idesc_o, (it > g0 || kk > 0) ? 1u : 0u);
+            const uint32_t vbase = sV + vs * C::kTileBytes;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (!mbar_wait(bar_p_full(h), it & 1, abort_flag, p.status)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              // half h: keys 64h .. 64h+63 of the iteration = 16-key steps 4h .. 4h+3
+              const int kend = min(2 * ns, 4 * h + 4);
+              for (int kk = 4 * h; kk < kend; ++kk) {
+                const uint64_t a = smem_desc_sw128(sP + h * kPanelBytes + (kk & 3) * 32, 16, 1024);
+                const uint64_t b =
+                    smem_desc_sw128(vbase + kk * 16 * kPanelRowBytes, kPanelBytes, 1024);
+                mma_bf16_ss(tmem_base + C::kOCol + 128 * h, a, b, idesc_o,
+                            (started[h] || kk > 4 * h) ? 1u : 0u);
+              }
+              if (kend > 4 * h) started[h] = true;
+              mma_commit(bar_o_done(h));
             }
-            mma_commit(bar_o_done);
-            mma_commit(bar_kv_empty(stage));
+            if (!ok) break;
+            mma_commit(bar_v_empty(vs));
           }
           ++it;
           if (last) break;
@@ -418,12 +508,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else {
-    // ======================================================= softmax / epilogue
-    const int wg = warp & 3;         // TMEM lane quarter owned by this warp
-    const int r = wg * 32 + lane;    // row within the tile
+  } else if (warp >= 4) {
+    // ======================================================= softmax / epilogue (warps 4..11)
+    const int half = (warp - 4) >> 2;   // key slots 2*half, 2*half+1
+    const int wg = warp & 3;            // TMEM lane quarter owned by this warp
+    const int r = wg * 32 + lane;       // row within the tile
     const uint32_t t_row = tmem_base + ((uint32_t)(wg * 32) << 16);
+    const uint32_t o_col = C::kOCol + 128 * half;
     const float sl2 = p.scale_log2;
+    float* xchg = reinterpret_cast<float*>(smem + C::kOffP);  // epilogue only: P is idle then
     uint32_t it = 0;
     int tl = 0;
     bool ok = true;
@@ -435,128 +528,166 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m = -INFINITY, l = 0.f;
       float lse_l2 = 0.f;
       if (!C::kAttn && i < p.n) lse_l2 = p.lse_in[(long long)bh * p.n + i] * 1.4426950408889634f;
-      const uint32_t g0 = it;
+      bool started = false;   // mirrors the MMA issuer: this half's O written in this tile
+      bool wrote_other = false;
       while (true) {
-        const int stage = it % C::kStages;
-        if (!warp_wait(bar_kv_full(stage), (it / C::kStages) & 1, abort_flag, p.status)) {
+        const int is = it % kInfoRing;
+        if (!warp_wait(bar_i_full(is), (it / kInfoRing) & 1, abort_flag, p.status)) {
           ok = false;
           break;
         }
-        const int ns = info[stage].nslots;
-        const int last = info[stage].last;
-        int kbs[kSlots], vld[kSlots];
+        const int ns = info[is].nslots;
+        const int last = info[is].last;
+        int kbs[2], vld[2];
 #pragma unroll
-        for (int s = 0; s < kSlots; ++s) {
-          kbs[s] = info[stage].kb[s];
-          vld[s] = (s < ns) && ((info[stage].own[s] >> wg) & 1);
+        for (int x = 0; x < 2; ++x) {
+          const int s = 2 * half + x;
+          kbs[x] = info[is].kb[s];
+          vld[x] = (s < ns) && ((info[is].own[s] >> wg) & 1);
         }
-        if (!C::kAttn) mbar_arrive(bar_kv_empty(stage));  // slot info consumed
+        mbar_arrive(bar_i_empty(is));
         if (!warp_wait(bar_s_full(it & 1), (it >> 1) & 1, abort_flag, p.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        uint32_t sr[kSlots][32];
+        uint32_t sr[2][32];
 #pragma unroll
-        for (int s = 0; s < kSlots; ++s)
-          if (vld[s]) tmem_ld32(t_row + (it & 1) * 128 + s * 32, sr[s]);
+        for (int x = 0; x < 2; ++x)
+          if (vld[x]) tmem_ld32(t_row + (it & 1) * 128 + (2 * half + x) * 32, sr[x]);
         tmem_wait_ld();
-#pragma unroll
-        for (int s = 0; s < kSlots; ++s) reg_fence32(sr[s]);
+        reg_fence(sr[0]);
+        reg_fence(sr[1]);
         tc_fence_before();
         mbar_arrive(bar_s_free(it & 1));
 
         if (!C::kAttn) {
           // ---------------- block mass: sum_j exp(s_ij*scale - lse_i) over the block, mean over rows
+          float acc[2];
 #pragma unroll
-          for (int s = 0; s < kSlots; ++s) {
-            if (!vld[s]) continue;
-            const bool diag = kbs[s] == qb;
-            float acc = 0.f;
+          for (int x = 0; x < 2; ++x) {
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+            if (vld[x]) {
+              if (kbs[x] == qb) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const float x = __uint_as_float(sr[s][c]);
-              const float e = fast_exp2(fmaf(x, sl2, -lse_l2));
-              acc += (diag && c > lane) ? 0.f : e;
+                for (int c = 0; c < 32; ++c) {
+                  const float e = fast_exp2(fmaf(__uint_as_float(sr[x][c]), sl2, -lse_l2));
+                  a4[c & 3] += (c > lane) ? 0.f : e;
+                }
+              } else {
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                  a4[c & 3] += fast_exp2(fmaf(__uint_as_float(sr[x][c]), sl2, -lse_l2));
+              }
             }
+            acc[x] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+          }
+          // the warp's 32 lanes are the 32 rows of query block qb: two interleaved butterflies
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (lane == 0)
-              p.mass[((long long)bh * p.nq + qb) * p.nq + kbs[s]] = acc * (1.0f / 32.0f);
+          for (int o = 16; o > 0; o >>= 1) {
+            acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], o);
+            acc[1] += __shfl_xor_sync(0xffffffffu, acc[1], o);
+          }
+          if (lane < 2) {
+            const float mine = lane == 0 ? acc[0] : acc[1];
+            const int kbl = lane == 0 ? kbs[0] : kbs[1];
+            const int v = lane == 0 ? vld[0] : vld[1];
+            if (v) p.mass[((long long)bh * p.nq + qb) * p.nq + kbl] = mine * (1.0f / 32.0f);
           }
         } else {
-          // ---------------- online softmax (log2 domain, lazily rescaled)
-          float mx = -INFINITY;
+          // ---------------- online softmax of this half (log2 domain, lazily rescaled)
 #pragma unroll
-          for (int s = 0; s < kSlots; ++s) {
-            const bool diag = kbs[s] == qb;
+          for (int x = 0; x < 2; ++x) {
+            if (vld[x] && kbs[x] == qb) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              float x = vld[s] ? __uint_as_float(sr[s][c]) * sl2 : -INFINITY;
-              if (diag && c > lane) x = -INFINITY;
-              sr[s][c] = __float_as_uint(x);
-              mx = fmaxf(mx, x);
+              for (int c = 0; c < 32; ++c)
+                if (c > lane) sr[x][c] = __float_as_uint(-INFINITY);
             }
           }
+          float mxa[8];
+#pragma unroll
+          for (int y = 0; y < 8; ++y) mxa[y] = -INFINITY;
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            if (vld[x]) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c)
+                mxa[c & 7] = fmaxf(mxa[c & 7], __uint_as_float(sr[x][c]));
+            }
+          }
+#pragma unroll
+          for (int y = 0; y < 4; ++y) mxa[y] = fmaxf(mxa[y], mxa[y + 4]);
+          const float mx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])) * sl2;
           const float m_new = fmaxf(m, mx);
           const bool need = m_new > m + 8.0f;   // true on the first finite score
           const bool warp_need = __any_sync(0xffffffffu, need);
           const float m_use = warp_need ? m_new : m;
           const float alpha = (warp_need && m != -INFINITY) ? fast_exp2(m - m_use) : 1.0f;
-          float rs = 0.f;
+          const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;  // all scores are -inf then
+          float rsa[8];
 #pragma unroll
-          for (int s = 0; s < kSlots; ++s) {
+          for (int y = 0; y < 8; ++y) rsa[y] = 0.f;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const float x = __uint_as_float(sr[s][c]);
-              const float e = (m_use == -INFINITY) ? 0.f : fast_exp2(x - m_use);
-              sr[s][c] = __float_as_uint(e);
-              rs += e;
+          for (int x = 0; x < 2; ++x) {
+            if (vld[x]) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                const float e = fast_exp2(fmaf(__uint_as_float(sr[x][c]), sl2, neg_m));
+                sr[x][c] = __float_as_uint(e);
+                rsa[c & 7] += e;
+              }
             }
           }
+#pragma unroll
+          for (int y = 0; y < 4; ++y) rsa[y] += rsa[y + 4];
+          const float rs = (rsa[0] + rsa[1]) + (rsa[2] + rsa[3]);
           l = l * alpha + rs;
           m = m_use;
-          // The previous PV must be done before P is overwritten or O rescaled.
-          if (it > g0 && !warp_wait(bar_o_done, (it - 1) & 1, abort_flag, p.status)) {
+          // This half's previous PV must be done before its P is overwritten or its O rescaled.
+          if (it > 0 && !warp_wait(bar_o_done(half), (it - 1) & 1, abort_flag, p.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          if (warp_need && it > g0) {
+          if (warp_need && started) {
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t o[32];
-              tmem_ld32(t_row + C::kOCol + c * 32, o);
+            for (int c = 0; c < D / 16; ++c) {
+              uint32_t o[16];
+              tmem_ld16(t_row + o_col + c * 16, o);
               tmem_wait_ld();
-              reg_fence32(o);
+              reg_fence(o);
 #pragma unroll
-              for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-              tmem_st32(t_row + C::kOCol + c * 32, o);
+              for (int y = 0; y < 16; ++y) o[y] = __float_as_uint(__uint_as_float(o[y]) * alpha);
+              tmem_st16(t_row + o_col + c * 16, o);
             }
             tmem_wait_st();
           }
-          // P (bf16) -> shared memory, K-major 128-byte swizzle, keys 0..127 in two panels.
+          // P (bf16) -> shared memory panel `half` (keys 64*half .. +63), 128-byte swizzle.
 #pragma unroll
-          for (int s = 0; s < kSlots; ++s) {
-            if (s >= ns) continue;
+          for (int x = 0; x < 2; ++x) {
+            if (2 * half + x >= ns) continue;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {   // 8 keys per 16-byte chunk
-              const int key0 = s * 32 + ch * 8;
-              const int pnl = key0 >> 6;
-              const int cc = (key0 & 63) >> 3;
-              uint32_t w0 = pack_bf16x2(__uint_as_float(sr[s][ch * 8 + 0]), __uint_as_float(sr[s][ch * 8 + 1]));
-              uint32_t w1 = pack_bf16x2(__uint_as_float(sr[s][ch * 8 + 2]), __uint_as_float(sr[s][ch * 8 + 3]));
-              uint32_t w2 = pack_bf16x2(__uint_as_float(sr[s][ch * 8 + 4]), __uint_as_float(sr[s][ch * 8 + 5]));
-              uint32_t w3 = pack_bf16x2(__uint_as_float(sr[s][ch * 8 + 6]), __uint_as_float(sr[s][ch * 8 + 7]));
-              const uint32_t addr = sP + pnl * kPanelBytes + r * kPanelRowBytes + ((cc ^ (r & 7)) << 4);
+              const int cc = x * 4 + ch;
+              uint32_t w0 = 0u, w1 = 0u, w2 = 0u, w3 = 0u;   // slots this warp does not own: P = 0
+              if (vld[x]) {
+                w0 = pack_bf16x2(__uint_as_float(sr[x][ch * 8 + 0]), __uint_as_float(sr[x][ch * 8 + 1]));
+                w1 = pack_bf16x2(__uint_as_float(sr[x][ch * 8 + 2]), __uint_as_float(sr[x][ch * 8 + 3]));
+                w2 = pack_bf16x2(__uint_as_float(sr[x][ch * 8 + 4]), __uint_as_float(sr[x][ch * 8 + 5]));
+                w3 = pack_bf16x2(__uint_as_float(sr[x][ch * 8 + 6]), __uint_as_float(sr[x][ch * 8 + 7]));
+              }
+              const uint32_t addr =
+                  sP + half * kPanelBytes + r * kPanelRowBytes + ((cc ^ (r & 7)) << 4);
               asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1),
                            "r"(w2), "r"(w3)
                            : "memory");
             }
           }
+          if (2 * ns > 4 * half) started = true;
+          if (2 * ns > 4 * (1 - half)) wrote_other = true;
           fence_proxy_async_smem();
           tc_fence_before();
-          mbar_arrive(bar_p_full);
+          mbar_arrive(bar_p_full(half));
         }
         ++it;
         if (last) break;
@@ -564,42 +695,71 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
 
       if (C::kAttn) {
-        // ---------------- epilogue: O / l -> bf16 -> smem (reuses the Q tile) -> TMA store
-        if (!warp_wait(bar_o_done, (it - 1) & 1, abort_flag, p.status)) {
+        // ---------------- epilogue: merge the halves, O -> bf16 -> smem (Q tile) -> TMA store
+        if (!warp_wait(bar_o_done(0), (it - 1) & 1, abort_flag, p.status) ||
+            !warp_wait(bar_o_done(1), (it - 1) & 1, abort_flag, p.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const float inv_l = l > 0.f ? 1.0f / l : 0.f;
+        // exchange (m, l) with the other half's thread of the same row (P buffer is idle now)
+        xchg[(half * 128 + r) * 2 + 0] = m;
+        xchg[(half * 128 + r) * 2 + 1] = l;
+        mbar_arrive(bar_merge);
+        if (!warp_wait(bar_merge, tl & 1, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        const float m_o = xchg[((1 - half) * 128 + r) * 2 + 0];
+        const float l_o = xchg[((1 - half) * 128 + r) * 2 + 1];
+        const float ma = half == 0 ? m : m_o, la = half == 0 ? l : l_o;
+        const float mb = half == 0 ? m_o : m, lb = half == 0 ? l_o : l;
+        const bool a_written = half == 0 ? started : wrote_other;
+        const bool b_written = half == 0 ? wrote_other : started;
+        const float mt = fmaxf(ma, mb);
+        const float sa = (la > 0.f) ? fast_exp2(ma - mt) : 0.f;
+        const float sb = (lb > 0.f) ? fast_exp2(mb - mt) : 0.f;
+        const float L = la * sa + lb * sb;
+        const float inv = L > 0.f ? 1.0f / L : 0.f;
+        const float ca = sa * inv, cb = sb * inv;
+        // this half writes output columns [half*D/2, (half+1)*D/2)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(t_row + C::kOCol + c * 32, o);
-          tmem_wait_ld();
-          reg_fence32(o);
+          const int col0 = half * (D / 2) + c * 16;
+          uint32_t oa[16], ob[16];
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            const int col0 = c * 32 + ch * 8;
-            const int pnl = col0 >> 6;
-            const int cc = (col0 & 63) >> 3;
+          for (int y = 0; y < 16; ++y) oa[y] = ob[y] = 0u;
+          if (a_written) tmem_ld16(t_row + C::kOCol + col0, oa);
+          if (b_written) tmem_ld16(t_row + C::kOCol + 128 + col0, ob);
+          tmem_wait_ld();
+          reg_fence(oa);
+          reg_fence(ob);
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            const int cabs = col0 + ch * 8;
+            const int pnl = cabs >> 6;
+            const int cc = (cabs & 63) >> 3;
             uint32_t w[4];
 #pragma unroll
-            for (int x = 0; x < 4; ++x)
-              w[x] = pack_bf16x2(__uint_as_float(o[ch * 8 + 2 * x]) * inv_l,
-                                 __uint_as_float(o[ch * 8 + 2 * x + 1]) * inv_l);
+            for (int y = 0; y < 4; ++y) {
+              const int e0 = ch * 8 + 2 * y;
+              const float v0 = __uint_as_float(oa[e0]) * ca + __uint_as_float(ob[e0]) * cb;
+              const float v1 = __uint_as_float(oa[e0 + 1]) * ca + __uint_as_float(ob[e0 + 1]) * cb;
+              w[y] = pack_bf16x2(v0, v1);
+            }
             const uint32_t addr = sQ + pnl * kPanelBytes + r * kPanelRowBytes + ((cc ^ (r & 7)) << 4);
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]),
                          "r"(w[2]), "r"(w[3])
                          : "memory");
           }
         }
-        if (p.lse != nullptr && i < p.n)
+        if (half == 0 && p.lse != nullptr && i < p.n)
           p.lse[(long long)bh * p.n + i] =
-              l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+              L > 0.f ? (mt + __log2f(L)) * 0.6931471805599453f : -INFINITY;
         tc_fence_before();
         fence_proxy_async_smem();
         mbar_arrive(bar_o_staged);
-        if (warp == 2 && lane == 0) {
+        if (warp == 4 && lane == 0) {
           if (!mbar_wait(bar_o_staged, tl & 1, abort_flag, p.status)) {
             ok = false;
           } else {
@@ -614,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) *abort_flag = 1;
       }
     }
-    if (C::kAttn && warp == 2 && lane == 0) bulk_wait_group0();
+    if (C::kAttn && warp == 4 && lane == 0) bulk_wait_group0();
   }
 
   tc_fence_before();

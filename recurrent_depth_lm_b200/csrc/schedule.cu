@@ -6,11 +6,14 @@
 // key blocks are a reusable GPU-resident CSR schedule (row offsets + active
 // block indices), built once after discovery.
 //
-// Three launches, one thread per row (bh, q):
-//   count : popcount of the row's admissible bits, block sums -> workspace
+// Three launches over blocks of kSchedThreads rows (bh, q):
+//   count : popcount of each row's admissible bits (thread per row), block sums
+//           -> workspace
 //   scan  : exclusive scan of the block sums (one CTA), total -> row_offsets[rows]
-//   emit  : block-local exclusive scan + block base -> row_offsets[row], then
-//           the set bits in ascending order -> col_idx (clamped to capacity).
+//   emit  : block-local exclusive scan + block base -> row_offsets[row]; then one
+//           warp per row writes its set bits in ascending order -> col_idx, each
+//           lane expanding one 32-bit word at its warp-scanned offset (clamped to
+//           capacity).
 
 #include <cstdint>
 
@@ -18,7 +21,8 @@
 
 namespace wise {
 
-constexpr int kSchedThreads = 1024;
+constexpr int kSchedThreads = 256;
+constexpr int kSchedWarps = kSchedThreads / 32;
 
 __device__ __forceinline__ uint32_t admissible_word(const uint32_t* ub, long long row, int W, int w,
                                                     int q) {
@@ -37,7 +41,7 @@ __device__ __forceinline__ int row_count(const uint32_t* ub, long long row, int 
   return c;
 }
 
-// Inclusive scan over the block's 1024 threads; returns the inclusive value, *total = block sum.
+// Inclusive scan over the block's kSchedThreads threads; returns the inclusive value, *total = block sum.
 __device__ __forceinline__ int block_inclusive_scan(int x, int* warp_sums, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -48,17 +52,17 @@ __device__ __forceinline__ int block_inclusive_scan(int x, int* warp_sums, int* 
   if (lane == 31) warp_sums[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int s = warp_sums[lane];
+    int s = lane < kSchedWarps ? warp_sums[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, s, o);
       if (lane >= o) s += y;
     }
-    warp_sums[lane] = s;
+    if (lane < kSchedWarps) warp_sums[lane] = s;
   }
   __syncthreads();
   if (warp > 0) x += warp_sums[warp - 1];
-  *total = warp_sums[31];
+  *total = warp_sums[kSchedWarps - 1];
   return x;
 }
 
@@ -96,22 +100,41 @@ __global__ void __launch_bounds__(kSchedThreads)
                       int32_t* __restrict__ row_offsets, int32_t* __restrict__ col_idx,
                       long long capacity, long long rows, int nq) {
   __shared__ int warp_sums[32];
+  __shared__ int row_off[kSchedThreads];
   const int W = (nq + 31) >> 5;
-  const long long row = (long long)blockIdx.x * kSchedThreads + threadIdx.x;
+  const long long row0 = (long long)blockIdx.x * kSchedThreads;
+  const long long row = row0 + threadIdx.x;
   const int c = row < rows ? row_count(ub, row, W, nq) : 0;
   int total;
   const int inc = block_inclusive_scan(c, warp_sums, &total);
-  if (row >= rows) return;
-  long long off = (long long)block_base[blockIdx.x] + inc - c;
-  row_offsets[row] = (int32_t)off;
-  const int q = (int)(row % nq);
-  for (int w = 0; w < W; ++w) {
-    uint32_t word = admissible_word(ub, row, W, w, q);
-    while (word != 0u) {
-      const int b = __ffs(word) - 1;
-      word &= word - 1u;
-      if (off < capacity) col_idx[off] = w * 32 + b;
-      ++off;
+  const int off = block_base[blockIdx.x] + inc - c;
+  row_off[threadIdx.x] = off;
+  if (row < rows) row_offsets[row] = off;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int rr = warp; rr < kSchedThreads; rr += kSchedWarps) {
+    const long long r = row0 + rr;
+    if (r >= rows) break;
+    const int q = (int)(r % nq);
+    long long pos = row_off[rr];
+    for (int w0 = 0; w0 < W; w0 += 32) {
+      const int w = w0 + lane;
+      uint32_t word = w < W ? admissible_word(ub, r, W, w, q) : 0u;
+      const int cnt = __popc(word);
+      int pre = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, pre, o);
+        if (lane >= o) pre += y;
+      }
+      long long at = pos + pre - cnt;
+      while (word != 0u) {
+        const int b = __ffs(word) - 1;
+        word &= word - 1u;
+        if (at < capacity) col_idx[at] = w * 32 + b;
+        ++at;
+      }
+      pos += __shfl_sync(0xffffffffu, pre, 31);
     }
   }
 }

@@ -1,0 +1,127 @@
+"""Full WISE trajectories on the GPU against the oracle, for every workload config.
+
+The GPU runs every head of the config through the same calls the benchmark
+times (WiseTrajectory: dense / dense+mass+select / schedule / sparse); the
+oracle recomputes sampled heads from the same seeded inputs.  Checked:
+dense O, block masses and per-step selections on window steps (bit-exact up to
+near-cut rows), union = OR of the step selections, schedule = CSR of the union
+(bit-exact), and late-step O against masked attention with the GPU's schedule.
+The 16K config also runs an eta = 1.0 trajectory whose late steps must equal
+dense causal attention.
+"""
+
+import os
+
+import numpy as np
+import pytest
+
+from oracle import wise_oracle as O
+from parity_utils import (MASS_TOL, bits_to_bool, check_csr, compare_o, compare_selection)
+from wise_inputs import CONFIGS, bf16_bits_to_f64, iter_steps
+from wise_inputs.generator import StepPool
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+
+def _dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def run_config(cfg, sample, check_steps, etas=(None,)):
+    """Run all heads of `cfg` on the GPU; return host copies for the sampled heads."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from recurrent_depth_lm_b200 import WiseTrajectory, ops
+    idx = [b * cfg.heads + h for (b, h) in sample]
+    trajs = {eta: WiseTrajectory(cfg.batch, cfg.heads, cfg.seqlen, cfg.head_dim, t_d=cfg.t_d,
+                                 window=cfg.window, eta=cfg.eta if eta is None else eta,
+                                 keep_step_bits=True) for eta in etas}
+    res = {eta: {"o": {}, "mass": {}, "bits": {}} for eta in etas}
+    workers = max(1, min(16, (os.cpu_count() or 2)))
+    with StepPool(cfg, workers=workers) as pool:
+        for t, q, k, v in pool:
+            dq, dk, dv = _dev(q), _dev(k), _dev(v)
+            for eta, tr in trajs.items():
+                o = tr.step(t, dq, dk, dv)
+                flat = lambda x: x.reshape(cfg.bh, *x.shape[2:])[idx]
+                if t in check_steps:
+                    res[eta]["o"][t] = flat(o).float().cpu().numpy()
+                if tr.in_window(t):
+                    res[eta]["mass"][t] = flat(tr.mass).cpu().numpy()
+                    res[eta]["bits"][t] = flat(tr.step_bits[t]).cpu().numpy()
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    for eta, tr in trajs.items():
+        ro = tr.row_offsets.cpu().numpy()
+        ci = tr.col_idx.cpu().numpy()
+        nq = cfg.nq
+        res[eta]["union"] = tr.union.reshape(cfg.bh, nq, -1)[idx].cpu().numpy()
+        res[eta]["sched"] = [(ro[i * nq:(i + 1) * nq + 1] - ro[i * nq],
+                              ci[ro[i * nq]:ro[(i + 1) * nq]]) for i in idx]
+        res[eta]["density"] = tr.density()
+    return res
+
+
+def check_config(cfg, sample, check_steps, etas=(None,)):
+    res = run_config(cfg, sample, check_steps, etas)
+    nq = cfg.nq
+    host = {t: (q, k, v) for t, q, k, v in iter_steps(cfg, heads=sample)}
+    report = {}
+    for eta in etas:
+        r = res[eta]
+        e = cfg.eta if eta is None else eta
+        exempt = 0
+        for si in range(len(sample)):
+            # window steps: mass and selection
+            step_sel = []
+            for t in range(cfg.window[0], cfg.window[1] + 1):
+                q, k, _ = (bf16_bits_to_f64(x[si]) for x in host[t])
+                r_ref = O.block_mass(q, k, cfg.scale)
+                assert np.abs(np.tril(r["mass"][t][si]) - r_ref).max() <= MASS_TOL
+                sel_gpu = bits_to_bool(r["bits"][t][si], nq)
+                exempt += compare_selection(sel_gpu, r_ref, e)
+                step_sel.append(sel_gpu)
+            union = bits_to_bool(r["union"][si], nq)
+            assert np.array_equal(union, O.temporal_union(step_sel))
+            ro, ci = r["sched"][si]
+            check_csr(ro, ci, union)
+            sup = O.support_from_csr(ro, ci, nq)
+            for t in check_steps:
+                q, k, v = (bf16_bits_to_f64(x[si]) for x in host[t])
+                if t <= cfg.t_d:
+                    ref, _ = O.causal_attention(q, k, v, cfg.scale)
+                else:
+                    ref, _ = O.masked_attention(q, k, v, sup, cfg.scale)
+                    if e >= 1.0:   # eta = 1 reproduces dense causal attention
+                        dense, _ = O.causal_attention(q, k, v, cfg.scale)
+                        compare_o(r["o"][t][si], dense, f"eta=1 step {t}")
+                compare_o(r["o"][t][si], ref, f"{cfg.name} head {sample[si]} step {t}")
+        report[eta] = {"exempt_rows": exempt, "density": r["density"]}
+    return report
+
+
+def test_trajectory_tiny_all_heads_all_steps():
+    cfg = CONFIGS["tiny"]
+    rep = check_config(cfg, [(0, 0), (0, 1)], check_steps=range(1, cfg.steps + 1))
+    assert rep[None]["exempt_rows"] <= 1
+
+
+def test_trajectory_1k():
+    cfg = CONFIGS["1k"]
+    check_config(cfg, [(0, 0), (0, 13), (0, 31)], check_steps=range(1, cfg.steps + 1))
+
+
+def test_trajectory_4k():
+    cfg = CONFIGS["4k"]
+    check_config(cfg, [(0, 0), (0, 21)], check_steps=[1, 9, 12, 13, 20, 32])
+
+
+def test_trajectory_2k_b4_h40_d96():
+    cfg = CONFIGS["2k_b4_h40_d96"]
+    check_config(cfg, [(0, 0), (2, 17), (3, 39)], check_steps=[1, 12, 13, 25, 32])
+
+
+def test_trajectory_16k_and_eta_one():
+    cfg = CONFIGS["16k"]
+    check_config(cfg, [(0, 5)], check_steps=[12, 13, 32], etas=(None, 1.0))

@@ -203,3 +203,70 @@ def generate_all_steps(cfg: WorkloadConfig, rank: int = 0, steps: int | None = N
         parts = [_head_all_steps(j) for j in jobs]
     arr = np.stack(parts, axis=2)  # [T, 3, BH, n, d]
     return arr.reshape(T, 3, cfg.batch, cfg.heads, cfg.seqlen, cfg.head_dim)
+
+
+def _pool_worker(conn, cfg, heads, rank, T):
+    streams = [HeadStream(cfg, b, h, rank) for (b, h) in heads]
+    n, d = cfg.seqlen, cfg.head_dim
+    for _ in range(T):
+        if conn.recv() is None:
+            break
+        out = np.empty((len(streams), 3, n, d), np.uint16)
+        for i, s in enumerate(streams):
+            out[i, 0], out[i, 1], out[i, 2] = s.next_step()
+        conn.send_bytes(out.tobytes())
+    conn.close()
+
+
+class StepPool:
+    """Step-by-step generation of all heads, spread over spawn-started processes.
+
+    Yields the same arrays as ``iter_steps(cfg)`` (every head owns its stream)
+    while bounding host memory to one step.  Use as a context manager.
+    """
+
+    def __init__(self, cfg: WorkloadConfig, workers: int, rank: int = 0, steps: int | None = None):
+        import multiprocessing as mp
+        self.cfg = cfg
+        self.T = cfg.steps if steps is None else steps
+        heads = all_heads(cfg)
+        workers = max(1, min(workers, len(heads)))
+        self.parts = [heads[i::workers] for i in range(workers)]
+        ctx = mp.get_context("spawn")
+        self.conns, self.procs = [], []
+        for part in self.parts:
+            a, b = ctx.Pipe()
+            p = ctx.Process(target=_pool_worker, args=(b, cfg, part, rank, self.T), daemon=True)
+            p.start()
+            self.conns.append(a)
+            self.procs.append(p)
+
+    def __iter__(self):
+        cfg = self.cfg
+        n, d = cfg.seqlen, cfg.head_dim
+        for t in range(1, self.T + 1):
+            for c in self.conns:
+                c.send(t)
+            full = np.empty((cfg.batch * cfg.heads, 3, n, d), np.uint16)
+            for wi, (c, part) in enumerate(zip(self.conns, self.parts)):
+                arr = np.frombuffer(c.recv_bytes(), np.uint16).reshape(len(part), 3, n, d)
+                full[wi::len(self.parts)] = arr
+            shp = (cfg.batch, cfg.heads, n, d)
+            yield t, full[:, 0].reshape(shp), full[:, 1].reshape(shp), full[:, 2].reshape(shp)
+
+    def close(self):
+        for c in self.conns:
+            try:
+                c.send(None)
+            except (BrokenPipeError, OSError):
+                pass
+        for p in self.procs:
+            p.join(timeout=10)
+            if p.is_alive():
+                p.kill()
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
