@@ -138,6 +138,34 @@ int wise_build_schedule(const uint32_t* union_bits, int32_t* row_offsets, int32_
                         size_t workspace_bytes, wise_shape_t shape, void* stream);
 
 /*
+ * wise_build_schedule without a caller-provided workspace.
+ *
+ * The WISE paper has no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory, e.g. code embedded in a host framework
+ * that owns every device allocation through its own pool, or a latency-bound
+ * serving loop where cudaMalloc (which can synchronise the device) is not
+ * allowed after start-up.  It computes exactly what wise_build_schedule
+ * computes, with the same arguments minus the workspace, and allocates
+ * nothing: its scan scratch is a fixed 16 KiB device array inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits.
+ *
+ * Limit      : batch * heads * seqlen / 32 <= 1,048,576 schedule rows; larger
+ *              shapes return WISE_ERR_WORKSPACE (use wise_build_schedule).
+ * Set-up     : the first call on each device looks up the array's device
+ *              address (with that device current); make that first call before
+ *              any stream capture.
+ * Sharing    : all calls on a device use the same array and it keeps the last
+ *              call's contents (nothing in it needs clearing: every entry read
+ *              is written first by the same call).  Calls whose kernels overlap
+ *              on the GPU, e.g. on unordered streams, race on it.
+ * Errors     : as wise_build_schedule, with WISE_ERR_WORKSPACE for the limit.
+ */
+int wise_build_schedule_static(const uint32_t* union_bits, int32_t* row_offsets, int32_t* col_idx,
+                               int64_t col_capacity, int64_t* nnz_out, wise_shape_t shape,
+                               void* stream);
+
+/*
  * Late-step block-sparse causal attention over a CSR schedule.
  *
  * Defines (WISE paper section 5.2, reuse mask R, and section 7.4): the dense

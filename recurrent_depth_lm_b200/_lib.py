@@ -52,6 +52,8 @@ _SIGNATURES = {
     "wise_build_schedule": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int64,
                                            ctypes.POINTER(ctypes.c_int64), _vp, ctypes.c_size_t,
                                            WiseShape, _vp]),
+    "wise_build_schedule_static": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int64,
+                                                  ctypes.POINTER(ctypes.c_int64), WiseShape, _vp]),
     "wise_sparse_attn": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int64, _vp,
                                         WiseShape, _vp]),
     "wise_device_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]),

@@ -163,6 +163,13 @@ int launch_attn(int mode, const void* q, const void* k, const void* v, void* o,
 
 }  // namespace
 
+namespace wise {
+// For entry points defined in other translation units of the library.
+int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
+int record_ok() { return ok(); }
+int validate_shape(const wise_shape_t& s) { return check_shape(s); }
+}  // namespace wise
+
 extern "C" {
 
 int wise_full_attn_mass(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "wise.h"
+
 namespace wise {
 
 enum { kModeDense = 0, kModeSparse = 1, kModeMass = 2 };
@@ -36,5 +38,10 @@ size_t schedule_workspace_bytes(long long rows);
 cudaError_t launch_build_schedule(const uint32_t* union_bits, int32_t* row_offsets,
                                   int32_t* col_idx, long long capacity, void* workspace,
                                   long long rows, int nq, cudaStream_t stream);
+
+// Error recording and shape validation shared with entry points outside api.cu.
+int record_error(int code, const char* msg);
+int record_ok();
+int validate_shape(const wise_shape_t& s);
 
 }  // namespace wise
