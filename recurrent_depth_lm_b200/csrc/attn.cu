@@ -23,7 +23,9 @@
 // Shared memory (128-byte swizzle, 1024-byte aligned panels of 64 columns):
 //   Q tile [128 x d], K and V stage rings [128 keys x d], P [128 x 128] bf16.
 // Tensor memory: S double buffer (2 x 128 fp32 columns) + one O accumulator
-// per softmax half (2 x 128 columns).
+// per softmax half (2 x 128 columns).  Each half writes its P (bf16, two per
+// column) over the first 32 columns of its own 64-column part of the S buffer
+// it just read, and the PV MMA reads P from there (A operand in TMEM).
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -36,7 +38,7 @@ namespace wise {
 
 constexpr int kBM = 128;        // query rows per tile
 constexpr int kSlots = 4;       // key blocks per iteration
-constexpr int kThreads = 384;   // 12 warps
+constexpr int kThreads = 352;   // 11 warps
 constexpr int kPanelRowBytes = 128;                // 64 bf16 per swizzled row
 constexpr int kPanelBytes = kBM * kPanelRowBytes;  // one 128-row panel = 16 KB
 constexpr int kMaxWords = 16;   // schedule bitmask words per query block (nq <= 512)
@@ -54,15 +56,15 @@ struct Cfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kTileBytes;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
-  static constexpr int kOffP = kOffV + kVStages * kTileBytes;
-  static constexpr int kOffInfo = kOffP + (kAttn ? 2 * kPanelBytes : 0);
+  static constexpr int kOffX = kOffV + kVStages * kTileBytes;   // epilogue (m, l) exchange
+  static constexpr int kOffInfo = kOffX + (kAttn ? 2 * kBM * 8 : 0);
   static constexpr int kInfoBytes = 64;
   static constexpr int kOffMask = kOffInfo + kInfoRing * kInfoBytes;
   static constexpr int kOffBar = kOffMask + 4 * kMaxWords * 4;
   static constexpr int kVRing = kVStages > 0 ? kVStages : 1;  // barrier slots (mass mode: unused)
   // q_full, q_empty, k_full[K], k_empty[K], v_full[V], v_empty[V], info_full[I], info_empty[I],
-  // s_full[2], s_free[2], p_full[2], o_done[2], merge, o_staged, final, spare
-  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVRing + 2 * kInfoRing + 12;
+  // s_full[2], s_free[2], p_full[2 halves][2 S buffers], o_done[2], merge, o_staged, final
+  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVRing + 2 * kInfoRing + 14;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
   static constexpr uint32_t kTmemCols = kAttn ? 512 : 256;
@@ -195,10 +197,10 @@ __device__ __forceinline__ void decode_tile(int tile, int BH, int ntq, int& bh, 
 
 // ---------------------------------------------------------------- the kernel
 //
-// Warp roles (384 threads): warp 0 = Q/K TMA producer and slot-list writer;
+// Warp roles (352 threads): warp 0 = Q/K TMA producer and slot-list writer;
 // warp 1 = TMEM allocator + single-thread MMA issuer; warp 2 = V TMA producer;
-// warp 3 idle; warps 4..11 = softmax in two halves.  Half h (warps 4+4h ..
-// 7+4h) owns key slots 2h and 2h+1 of every iteration (S columns 64h..64h+63)
+// warps 3..10 = softmax in two halves.  Half h (warps 3+4h .. 6+4h) owns key
+// slots 2h and 2h+1 of every iteration (S columns 64h..64h+63)
 // and keeps its own online-softmax state (m, l) and its own O accumulator in
 // TMEM; the two partial results of a row are merged once, in the epilogue:
 //   O = (2^(m_a-m) O_a + 2^(m_b-m) O_b) / (2^(m_a-m) l_a + 2^(m_b-m) l_b).
@@ -222,7 +224,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sQ = smem_u32(smem + C::kOffQ);
   const uint32_t sK = smem_u32(smem + C::kOffK);
   const uint32_t sV = smem_u32(smem + C::kOffV);
-  const uint32_t sP = smem_u32(smem + C::kOffP);
   StageInfo* info = (StageInfo*)(smem + C::kOffInfo);
   uint32_t* tile_mask = (uint32_t*)(smem + C::kOffMask);
   const uint32_t bar0 = smem_u32(smem + C::kOffBar);
@@ -240,11 +241,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t barS = barI + 16 * kInfoRing;
   auto bar_s_full = [&](int b) { return barS + 8 * b; };
   auto bar_s_free = [&](int b) { return barS + 16 + 8 * b; };
-  auto bar_p_full = [&](int h) { return barS + 32 + 8 * h; };
-  auto bar_o_done = [&](int h) { return barS + 48 + 8 * h; };
-  const uint32_t bar_merge = barS + 64;
-  const uint32_t bar_o_staged = barS + 72;
-  const uint32_t bar_final = barS + 80;
+  // one p_full per (half, S buffer): the softmax may run an iteration ahead of the
+  // MMA issuer, so a single barrier per half could complete two phases unobserved
+  auto bar_p_full = [&](int h, int b) { return barS + 32 + 16 * h + 8 * b; };
+  // one o_done per S buffer: arrives when both halves' PV of an iteration using that
+  // buffer has completed (phase index = iteration >> 1)
+  auto bar_o_done = [&](int b) { return barS + 64 + 8 * b; };
+  const uint32_t bar_merge = barS + 80;
+  const uint32_t bar_o_staged = barS + 88;
+  const uint32_t bar_final = barS + 96;
   volatile int* abort_flag = (volatile int*)(smem + C::kOffMisc);
   uint32_t* tmem_slot = (uint32_t*)(smem + C::kOffMisc + 4);
 
@@ -270,7 +275,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_s_full(b), 1);
       mbar_init(bar_s_free(b), kSoftmaxThreads);
-      mbar_init(bar_p_full(b), kSoftmaxThreads / 2);
+      mbar_init(bar_p_full(0, b), kSoftmaxThreads / 2);
+      mbar_init(bar_p_full(1, b), kSoftmaxThreads / 2);
       mbar_init(bar_o_done(b), 1);
     }
     mbar_init(bar_merge, kSoftmaxThreads);
@@ -427,8 +433,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_qk = [&](uint32_t j, int& ns, int& last) -> bool {
         const int ks = j % NK;
         if (!mbar_wait(bar_k_full(ks), (j / NK) & 1, abort_flag, p.status)) return false;
-        if (j >= 2 && !mbar_wait(bar_s_free(j & 1), ((j >> 1) - 1) & 1, abort_flag, p.status))
-          return false;
+        if (j >= 2) {
+          // S buffer j&1 still holds S_{j-2} (mass mode) or P_{j-2} (attention modes)
+          if (!C::kAttn) {
+            if (!mbar_wait(bar_s_free(j & 1), ((j >> 1) - 1) & 1, abort_flag, p.status))
+              return false;
+          } else if (!mbar_wait(bar_o_done(j & 1), ((j >> 1) - 1) & 1, abort_flag, p.status)) {
+            return false;   // PV_{j-2} has read its P out of buffer j&1
+          }
+        }
         tc_fence_after();
         ns = info[j % kInfoRing].nslots;
         last = info[j % kInfoRing].last;
@@ -473,24 +486,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t vbase = sV + vs * C::kTileBytes;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              if (!mbar_wait(bar_p_full(h), it & 1, abort_flag, p.status)) {
+              if (!mbar_wait(bar_p_full(h, it & 1), (it >> 1) & 1, abort_flag, p.status)) {
                 ok = false;
                 break;
               }
               tc_fence_after();
-              // half h: keys 64h .. 64h+63 of the iteration = 16-key steps 4h .. 4h+3
+              // half h: keys 64h .. 64h+63 of the iteration = 16-key steps 4h .. 4h+3;
+              // its P sits in TMEM columns 64h .. 64h+31 of S buffer it&1 (8 per step)
               const int kend = min(2 * ns, 4 * h + 4);
+              const uint32_t p_tmem = tmem_base + (it & 1) * 128 + 64 * h;
               for (int kk = 4 * h; kk < kend; ++kk) {
-                const uint64_t a = smem_desc_sw128(sP + h * kPanelBytes + (kk & 3) * 32, 16, 1024);
                 const uint64_t b =
                     smem_desc_sw128(vbase + kk * 16 * kPanelRowBytes, kPanelBytes, 1024);
-                mma_bf16_ss(tmem_base + C::kOCol + 128 * h, a, b, idesc_o,
+                mma_bf16_ts(tmem_base + C::kOCol + 128 * h, p_tmem + (kk - 4 * h) * 8, b, idesc_o,
                             (started[h] || kk > 4 * h) ? 1u : 0u);
               }
               if (kend > 4 * h) started[h] = true;
-              mma_commit(bar_o_done(h));
             }
             if (!ok) break;
+            mma_commit(bar_o_done(it & 1));
             mma_commit(bar_v_empty(vs));
           }
           ++it;
@@ -508,15 +522,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= 4) {
-    // ======================================================= softmax / epilogue (warps 4..11)
-    const int half = (warp - 4) >> 2;   // key slots 2*half, 2*half+1
+  } else {
+    // ======================================================= softmax / epilogue (warps 3..10)
+    const int half = (warp - 3) >> 2;   // key slots 2*half, 2*half+1
     const int wg = warp & 3;            // TMEM lane quarter owned by this warp
     const int r = wg * 32 + lane;       // row within the tile
     const uint32_t t_row = tmem_base + ((uint32_t)(wg * 32) << 16);
     const uint32_t o_col = C::kOCol + 128 * half;
     const float sl2 = p.scale_log2;
-    float* xchg = reinterpret_cast<float*>(smem + C::kOffP);  // epilogue only: P is idle then
+    float* xchg = reinterpret_cast<float*>(smem + C::kOffX);
     uint32_t it = 0;
     int tl = 0;
     bool ok = true;
@@ -558,10 +572,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         reg_fence(sr[0]);
         reg_fence(sr[1]);
-        tc_fence_before();
-        mbar_arrive(bar_s_free(it & 1));
-
         if (!C::kAttn) {
+          tc_fence_before();
+          mbar_arrive(bar_s_free(it & 1));
           // ---------------- block mass: sum_j exp(s_ij*scale - lse_i) over the block, mean over rows
           float acc[2];
 #pragma unroll
@@ -596,6 +609,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {
           // ---------------- online softmax of this half (log2 domain, lazily rescaled)
+          // Slot validity and the diagonal are warp-uniform branches.  Packed f32x2
+          // FMA/ADD and 3-input max keep the instruction count per element low.
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
             if (vld[x] && kbs[x] == qb) {
@@ -604,52 +619,62 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (c > lane) sr[x][c] = __float_as_uint(-INFINITY);
             }
           }
-          float mxa[8];
-#pragma unroll
-          for (int y = 0; y < 8; ++y) mxa[y] = -INFINITY;
+          float mxa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
             if (vld[x]) {
 #pragma unroll
-              for (int c = 0; c < 32; ++c)
-                mxa[c & 7] = fmaxf(mxa[c & 7], __uint_as_float(sr[x][c]));
+              for (int c = 0; c < 32; c += 8) {
+#pragma unroll
+                for (int y = 0; y < 4; ++y)
+                  mxa[y] = max3(mxa[y], __uint_as_float(sr[x][c + 2 * y]),
+                                __uint_as_float(sr[x][c + 2 * y + 1]));
+              }
             }
           }
-#pragma unroll
-          for (int y = 0; y < 4; ++y) mxa[y] = fmaxf(mxa[y], mxa[y + 4]);
-          const float mx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])) * sl2;
+          const float mx = max3(mxa[0], mxa[1], fmaxf(mxa[2], mxa[3])) * sl2;
           const float m_new = fmaxf(m, mx);
           const bool need = m_new > m + 8.0f;   // true on the first finite score
           const bool warp_need = __any_sync(0xffffffffu, need);
           const float m_use = warp_need ? m_new : m;
           const float alpha = (warp_need && m != -INFINITY) ? fast_exp2(m - m_use) : 1.0f;
           const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;  // all scores are -inf then
-          float rsa[8];
-#pragma unroll
-          for (int y = 0; y < 8; ++y) rsa[y] = 0.f;
+          const uint64_t sc2 = f2(sl2, sl2), nm2 = f2(neg_m, neg_m);
+          uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
+          // P of slot x, keys 2c' and 2c'+1 as one bf16 pair, goes to sr[x][c'] (already consumed)
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
             if (vld[x]) {
 #pragma unroll
-              for (int c = 0; c < 32; ++c) {
-                const float e = fast_exp2(fmaf(__uint_as_float(sr[x][c]), sl2, neg_m));
-                sr[x][c] = __float_as_uint(e);
-                rsa[c & 7] += e;
+              for (int c = 0; c < 32; c += 2) {
+                float t0, t1;
+                f2_split(fma2(f2(__uint_as_float(sr[x][c]), __uint_as_float(sr[x][c + 1])), sc2, nm2),
+                         t0, t1);
+                const float e0 = fast_exp2(t0), e1 = fast_exp2(t1);
+                rs2[(c >> 1) & 3] = add2(rs2[(c >> 1) & 3], f2(e0, e1));
+                sr[x][c >> 1] = pack_bf16x2(e0, e1);
               }
+            } else {
+#pragma unroll
+              for (int c = 0; c < 16; ++c) sr[x][c] = 0u;   // not this warp's block: P = 0
             }
           }
-#pragma unroll
-          for (int y = 0; y < 4; ++y) rsa[y] += rsa[y + 4];
-          const float rs = (rsa[0] + rsa[1]) + (rsa[2] + rsa[3]);
+          float rs;
+          {
+            const uint64_t t = add2(add2(rs2[0], rs2[1]), add2(rs2[2], rs2[3]));
+            float lo, hi;
+            f2_split(t, lo, hi);
+            rs = lo + hi;
+          }
           l = l * alpha + rs;
           m = m_use;
-          // This half's previous PV must be done before its P is overwritten or its O rescaled.
-          if (it > 0 && !warp_wait(bar_o_done(half), (it - 1) & 1, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
           if (warp_need && started) {
+            // O of this half is rescaled in place: its previous PV must have finished.
+            if (!warp_wait(bar_o_done((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
 #pragma unroll
             for (int c = 0; c < D / 16; ++c) {
               uint32_t o[16];
@@ -660,34 +685,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int y = 0; y < 16; ++y) o[y] = __float_as_uint(__uint_as_float(o[y]) * alpha);
               tmem_st16(t_row + o_col + c * 16, o);
             }
-            tmem_wait_st();
           }
-          // P (bf16) -> shared memory panel `half` (keys 64*half .. +63), 128-byte swizzle.
-#pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            if (2 * half + x >= ns) continue;
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {   // 8 keys per 16-byte chunk
-              const int cc = x * 4 + ch;
-              uint32_t w0 = 0u, w1 = 0u, w2 = 0u, w3 = 0u;   // slots this warp does not own: P = 0
-              if (vld[x]) {
-                w0 = pack_bf16x2(__uint_as_float(sr[x][ch * 8 + 0]), __uint_as_float(sr[x][ch * 8 + 1]));
-                w1 = pack_bf16x2(__uint_as_float(sr[x][ch * 8 + 2]), __uint_as_float(sr[x][ch * 8 + 3]));
-                w2 = pack_bf16x2(__uint_as_float(sr[x][ch * 8 + 4]), __uint_as_float(sr[x][ch * 8 + 5]));
-                w3 = pack_bf16x2(__uint_as_float(sr[x][ch * 8 + 6]), __uint_as_float(sr[x][ch * 8 + 7]));
-              }
-              const uint32_t addr =
-                  sP + half * kPanelBytes + r * kPanelRowBytes + ((cc ^ (r & 7)) << 4);
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1),
-                           "r"(w2), "r"(w3)
-                           : "memory");
-            }
-          }
+          // P -> TMEM over the first 32 columns of this half's part of S buffer it&1
+          tmem_st32_halves(t_row + (it & 1) * 128 + 64 * half, sr[0], sr[1]);
+          tmem_wait_st();
           if (2 * ns > 4 * half) started = true;
           if (2 * ns > 4 * (1 - half)) wrote_other = true;
-          fence_proxy_async_smem();
           tc_fence_before();
-          mbar_arrive(bar_p_full(half));
+          mbar_arrive(bar_p_full(half, it & 1));
         }
         ++it;
         if (last) break;
@@ -696,8 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       if (C::kAttn) {
         // ---------------- epilogue: merge the halves, O -> bf16 -> smem (Q tile) -> TMA store
-        if (!warp_wait(bar_o_done(0), (it - 1) & 1, abort_flag, p.status) ||
-            !warp_wait(bar_o_done(1), (it - 1) & 1, abort_flag, p.status)) {
+        if (!warp_wait(bar_o_done((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, p.status)) {
           ok = false;
           break;
         }
@@ -759,7 +763,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         fence_proxy_async_smem();
         mbar_arrive(bar_o_staged);
-        if (warp == 4 && lane == 0) {
+        if (warp == 3 && lane == 0) {
           if (!mbar_wait(bar_o_staged, tl & 1, abort_flag, p.status)) {
             ok = false;
           } else {
@@ -774,7 +778,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) *abort_flag = 1;
       }
     }
-    if (C::kAttn && warp == 4 && lane == 0) bulk_wait_group0();
+    if (C::kAttn && warp == 3 && lane == 0) bulk_wait_group0();
   }
 
   tc_fence_before();
