@@ -223,6 +223,7 @@ class TrajectoryRunner:
     def launches_per_trajectory(self) -> int:
         cfg = self.cfg
         nwin = cfg.window[1] - cfg.window[0] + 1
+        # dense steps: 1 kernel; window steps: attention + mass + select; schedule: 3
         return (cfg.t_d - nwin) + 3 * nwin + 3 + (cfg.steps - cfg.t_d)
 
     def run(self, q, k, v, events=None):
@@ -241,7 +242,8 @@ class TrajectoryRunner:
             if t <= cfg.t_d:
                 if tr.in_window(t):
                     a = ev() if events is not None else None
-                    ops.full_attn_mass(qt, kt, vt, o=self.o, lse=tr.lse, mass=tr.mass)
+                    ops.full_attn_mass(qt, kt, vt, o=self.o, lse=tr.lse, mass=tr.mass,
+                                       workspace=tr.mass_ws)
                     b = ev() if events is not None else None
                     ops.select_union(tr.mass, tr.union, cfg.eta, head_dim=cfg.head_dim)
                     c = ev() if events is not None else None

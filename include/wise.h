@@ -72,18 +72,28 @@ typedef struct wise_shape {
  * and, when `mass` is non-NULL, the block mass of section 5.1:
  *   mass[bh][q][b] = (1/32) sum_{i in block q} sum_{j in block b} A_ij,  b <= q.
  *
- * q, k, v : bf16 [B, H, n, d] inputs.
- * o       : bf16 [B, H, n, d] output.
- * lse     : fp32 [B, H, n] output, natural-log row normaliser
- *           lse_i = log sum_{j<=i} exp(s_ij * scale); may be NULL unless
- *           mass is requested (the mass pass reads it back).
- * mass    : fp32 [B, H, nq, nq] output or NULL.  Only entries b <= q are
- *           written; entries b > q are left untouched.
- * Errors  : WISE_ERR_ARG (q/k/v/o NULL, mass without lse), WISE_ERR_SHAPE,
- *           WISE_ERR_ALIGN, WISE_ERR_CUDA.
+ * q, k, v   : bf16 [B, H, n, d] inputs.
+ * o         : bf16 [B, H, n, d] output.
+ * lse       : fp32 [B, H, n] output, natural-log row normaliser
+ *             lse_i = log sum_{j<=i} exp(s_ij * scale); may be NULL unless
+ *             mass is requested.
+ * mass      : fp32 [B, H, nq, nq] output or NULL.  Only entries b <= q are
+ *             written; entries b > q are left untouched.
+ * workspace : device scratch for the one-pass mass, or NULL.  With at least
+ *             wise_mass_workspace_bytes(shape) bytes the attention kernel also
+ *             records every row's per-key-block log-sum-exp and a light kernel
+ *             turns them into block masses; with NULL the mass is computed by a
+ *             second pass that recomputes Q K^T.  Ignored when mass is NULL.
+ * Errors    : WISE_ERR_ARG (q/k/v/o NULL, mass without lse), WISE_ERR_SHAPE,
+ *             WISE_ERR_ALIGN, WISE_ERR_WORKSPACE (non-NULL but too small),
+ *             WISE_ERR_CUDA.
  */
 int wise_full_attn_mass(const void* q, const void* k, const void* v, void* o, float* lse,
-                        float* mass, wise_shape_t shape, void* stream);
+                        float* mass, void* workspace, size_t workspace_bytes, wise_shape_t shape,
+                        void* stream);
+
+/* Workspace bytes of the one-pass block mass: B * H * nq * n * 4. */
+size_t wise_mass_workspace_bytes(wise_shape_t shape);
 
 /*
  * Per-step cumulative-eta block support, OR-ed into the working set.

@@ -45,7 +45,9 @@ class WiseError(RuntimeError):
 
 _vp = ctypes.c_void_p
 _SIGNATURES = {
-    "wise_full_attn_mass": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, WiseShape, _vp]),
+    "wise_full_attn_mass": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
+                                           WiseShape, _vp]),
+    "wise_mass_workspace_bytes": (ctypes.c_size_t, [WiseShape]),
     "wise_select_union": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_float, WiseShape, _vp]),
     "wise_schedule_workspace_bytes": (ctypes.c_size_t, [WiseShape]),
     "wise_schedule_max_nnz": (ctypes.c_int64, [WiseShape]),

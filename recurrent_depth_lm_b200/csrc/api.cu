@@ -173,7 +173,8 @@ int validate_shape(const wise_shape_t& s) { return check_shape(s); }
 extern "C" {
 
 int wise_full_attn_mass(const void* q, const void* k, const void* v, void* o, float* lse,
-                        float* mass, wise_shape_t shape, void* stream) {
+                        float* mass, void* workspace, size_t workspace_bytes, wise_shape_t shape,
+                        void* stream) {
   int rc = check_shape(shape);
   if (rc) return rc;
   if (!q || !k || !v || !o) return fail(WISE_ERR_ARG, "q, k, v and o must be non-NULL");
@@ -182,11 +183,23 @@ int wise_full_attn_mass(const void* q, const void* k, const void* v, void* o, fl
     return fail(WISE_ERR_ALIGN, "q, k, v, o must be 16-byte aligned");
   if ((lse && !aligned16(lse)) || (mass && !aligned16(mass)))
     return fail(WISE_ERR_ALIGN, "lse and mass must be 16-byte aligned");
+  const bool one_pass = mass && workspace;
+  if (one_pass) {
+    const size_t need = wise_mass_workspace_bytes(shape);
+    if (workspace_bytes < need)
+      return fail(WISE_ERR_WORKSPACE, "mass workspace of %zu bytes required", need);
+    if (!aligned16(workspace)) return fail(WISE_ERR_ALIGN, "workspace must be 16-byte aligned");
+  }
   wise::AttnParams p{};
   p.lse = lse;
+  p.blse = one_pass ? static_cast<float*>(workspace) : nullptr;
   rc = launch_attn(wise::kModeDense, q, k, v, o, p, shape, stream);
   if (rc) return rc;
-  if (mass) {
+  if (one_pass) {
+    cudaError_t e = wise::launch_mass_from_blse(p.blse, lse, mass, shape.batch * shape.heads,
+                                                shape.seqlen, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "mass launch");
+  } else if (mass) {
     wise::AttnParams pm{};
     pm.lse_in = lse;
     pm.mass = mass;
@@ -194,6 +207,12 @@ int wise_full_attn_mass(const void* q, const void* k, const void* v, void* o, fl
     if (rc) return rc;
   }
   return ok();
+}
+
+size_t wise_mass_workspace_bytes(wise_shape_t shape) {
+  if (check_shape(shape)) return 0;
+  const size_t nq = shape.seqlen / 32;
+  return (size_t)shape.batch * shape.heads * nq * shape.seqlen * sizeof(float);
 }
 
 int wise_select_union(const float* mass, uint32_t* union_bits, uint32_t* step_bits, float eta,

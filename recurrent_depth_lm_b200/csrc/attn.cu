@@ -640,31 +640,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float alpha = (warp_need && m != -INFINITY) ? fast_exp2(m - m_use) : 1.0f;
           const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;  // all scores are -inf then
           const uint64_t sc2 = f2(sl2, sl2), nm2 = f2(neg_m, neg_m);
-          uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
+          float ps[2] = {0.f, 0.f};   // per-slot sums of this row's probabilities
           // P of slot x, keys 2c' and 2c'+1 as one bf16 pair, goes to sr[x][c'] (already consumed)
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
             if (vld[x]) {
+              uint64_t rs2[2] = {0ull, 0ull};
 #pragma unroll
               for (int c = 0; c < 32; c += 2) {
                 float t0, t1;
                 f2_split(fma2(f2(__uint_as_float(sr[x][c]), __uint_as_float(sr[x][c + 1])), sc2, nm2),
                          t0, t1);
                 const float e0 = fast_exp2(t0), e1 = fast_exp2(t1);
-                rs2[(c >> 1) & 3] = add2(rs2[(c >> 1) & 3], f2(e0, e1));
+                rs2[(c >> 1) & 1] = add2(rs2[(c >> 1) & 1], f2(e0, e1));
                 sr[x][c >> 1] = pack_bf16x2(e0, e1);
               }
+              float lo, hi;
+              f2_split(add2(rs2[0], rs2[1]), lo, hi);
+              ps[x] = lo + hi;
             } else {
 #pragma unroll
               for (int c = 0; c < 16; ++c) sr[x][c] = 0u;   // not this warp's block: P = 0
             }
           }
-          float rs;
-          {
-            const uint64_t t = add2(add2(rs2[0], rs2[1]), add2(rs2[2], rs2[3]));
-            float lo, hi;
-            f2_split(t, lo, hi);
-            rs = lo + hi;
+          const float rs = ps[0] + ps[1];
+          if (MODE == kModeDense && p.blse != nullptr) {
+            // block log-sum-exp of this row over each owned key block, log2 domain:
+            // blse = m + log2(sum_j 2^(s_ij*scale*log2e - m)); the mass pass turns it into
+            // block mass with the final lse.  Layout [bh][key block][row]: 32 lanes store
+            // 32 consecutive floats.
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+              if (vld[x])
+                p.blse[((long long)bh * p.nq + kbs[x]) * p.n + i] =
+                    ps[x] > 0.f ? m_use + __log2f(ps[x]) : -INFINITY;
+            }
           }
           l = l * alpha + rs;
           m = m_use;

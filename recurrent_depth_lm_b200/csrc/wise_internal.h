@@ -20,6 +20,7 @@ struct AttnParams {
   float* lse;           // [BH, n] output (dense / sparse), nullable
   const float* lse_in;  // [BH, n] input (mass mode)
   float* mass;          // [BH, nq, nq] output (mass mode)
+  float* blse;          // [BH, nq, n] block log2-sum-exp side output (dense mode), nullable
   const int32_t* row_offsets;  // sparse mode
   const int32_t* col_idx;      // sparse mode
   long long col_count;         // sparse mode: valid entries of col_idx
@@ -30,6 +31,10 @@ cudaError_t launch_attention(int mode, int d, const CUtensorMap& tq, const CUten
                              const CUtensorMap& tv, const CUtensorMap& to, const AttnParams& p,
                              int grid, cudaStream_t stream);
 int attention_smem_bytes(int mode, int d);
+
+// mass[bh][q][b] = (1/32) sum_{i in q} 2^(blse[bh][b][i] - lse[bh][i] * log2 e), b <= q
+cudaError_t launch_mass_from_blse(const float* blse, const float* lse, float* mass, int BH,
+                                  int n, cudaStream_t stream);
 
 cudaError_t launch_select_union(const float* mass, uint32_t* union_bits, uint32_t* step_bits,
                                 float eta, int BH, int nq, cudaStream_t stream);

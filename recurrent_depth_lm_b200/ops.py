@@ -48,20 +48,34 @@ def words_per_row(nq: int) -> int:
 
 
 def full_attn_mass(q, k, v, *, with_mass: bool = False, o=None, lse=None, mass=None,
-                   scale=None, stream=None):
-    """Dense causal attention (+ block mass).  Returns (o, lse, mass)."""
+                   workspace=None, one_pass: bool = True, scale=None, stream=None):
+    """Dense causal attention (+ block mass).  Returns (o, lse, mass).
+
+    With mass requested and ``one_pass`` (default), the block mass comes from the
+    per-key-block log-sum-exps the attention kernel records in ``workspace``
+    (allocated here if not given); ``one_pass=False`` uses the two-pass path.
+    """
     b, h, n, d = q.shape
     if o is None:
         o = torch.empty_like(q)
     _check_qkv(q, k, v, o)
     if with_mass and mass is None:
         mass = torch.empty(b, h, n // BLOCK, n // BLOCK, dtype=torch.float32, device=q.device)
-    if (with_mass or mass is not None) and lse is None:
+    if mass is not None and lse is None:
         lse = torch.empty(b, h, n, dtype=torch.float32, device=q.device)
+    if mass is not None and one_pass and workspace is None:
+        workspace = mass_workspace(b, h, n, d, q.device)
+    ws = workspace if (mass is not None and one_pass) else None
     rc = lib.wise_full_attn_mass(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(mass),
+                                 _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                  shape_of(q, scale), _stream(stream))
     check(rc, "wise_full_attn_mass")
     return o, lse, mass
+
+
+def mass_workspace(b: int, h: int, n: int, head_dim: int, device) -> torch.Tensor:
+    nbytes = lib.wise_mass_workspace_bytes(WiseShape(b, h, n, head_dim, 0.0))
+    return torch.empty(max(1, nbytes // 4), dtype=torch.float32, device=device)
 
 
 def select_union(mass, union_bits, eta: float, *, step_bits=None, head_dim: int = 128,

@@ -33,6 +33,8 @@ class WiseTrajectory:
         self.lse = torch.empty(batch, heads, seqlen, dtype=torch.float32, device=dev)
         self.mass = torch.empty(batch, heads, self.nq, self.nq, dtype=torch.float32, device=dev)
         self.union = ops.new_bitmask(batch, heads, self.nq, dev)
+        # per-(row, key block) log-sum-exps of the one-pass block mass (window steps)
+        self.mass_ws = ops.mass_workspace(batch, heads, seqlen, head_dim, dev)
         self.step_bits = {}
         self.keep_step_bits = keep_step_bits
         self.row_offsets = torch.empty(batch * heads * self.nq + 1, dtype=torch.int32, device=dev)
@@ -54,7 +56,8 @@ class WiseTrajectory:
         if t <= self.t_d:
             if self.in_window(t):
                 o, _, _ = ops.full_attn_mass(q, k, v, o=o, lse=self.lse, mass=self.mass,
-                                             scale=self.scale, stream=stream)
+                                             workspace=self.mass_ws, scale=self.scale,
+                                             stream=stream)
                 sb = None
                 if self.keep_step_bits:
                     sb = torch.empty_like(self.union)

@@ -49,7 +49,8 @@ def shape(lib, b=1, h=2, n=256, d=64, s=0.0):
 def test_bad_shapes_rejected(lib, b, h, n, d):
     L = lib.lib
     fake = 1 << 20
-    rc = L.wise_full_attn_mass(fake, fake, fake, fake, None, None, shape(lib, b, h, n, d), None)
+    rc = L.wise_full_attn_mass(fake, fake, fake, fake, None, None, None, 0, shape(lib, b, h, n, d),
+                               None)
     assert rc == lib.WISE_ERR_SHAPE, lib.last_error()
     rc = L.wise_sparse_attn(fake, fake, fake, fake, fake, fake, 1, None, shape(lib, b, h, n, d), None)
     assert rc == lib.WISE_ERR_SHAPE
@@ -59,9 +60,13 @@ def test_bad_shapes_rejected(lib, b, h, n, d):
 def test_null_and_alignment_rejected(lib):
     L = lib.lib
     s = shape(lib)
-    assert L.wise_full_attn_mass(None, 16, 16, 16, None, None, s, None) == lib.WISE_ERR_ARG
-    assert L.wise_full_attn_mass(16, 16, 16, 16, None, 16, s, None) == lib.WISE_ERR_ARG  # mass w/o lse
-    assert L.wise_full_attn_mass(18, 16, 16, 16, None, None, s, None) == lib.WISE_ERR_ALIGN
+    assert L.wise_full_attn_mass(None, 16, 16, 16, None, None, None, 0, s, None) == lib.WISE_ERR_ARG
+    # mass without lse
+    assert L.wise_full_attn_mass(16, 16, 16, 16, None, 16, None, 0, s, None) == lib.WISE_ERR_ARG
+    assert L.wise_full_attn_mass(18, 16, 16, 16, None, None, None, 0, s, None) == lib.WISE_ERR_ALIGN
+    # workspace given but too small
+    assert L.wise_full_attn_mass(16, 16, 16, 16, 16, 16, 16, 8, s, None) == lib.WISE_ERR_WORKSPACE
+    assert L.wise_mass_workspace_bytes(s) == 1 * 2 * 8 * 256 * 4
     assert L.wise_sparse_attn(16, 16, 16, 16, None, 16, 1, None, s, None) == lib.WISE_ERR_ARG
     assert L.wise_sparse_attn(16, 16, 16, 16, 16, 16, -1, None, s, None) == lib.WISE_ERR_ARG
     assert L.wise_sparse_attn(16, 16, 24, 16, 16, 16, 1, None, s, None) == lib.WISE_ERR_ALIGN

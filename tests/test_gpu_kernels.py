@@ -44,11 +44,14 @@ def dev_f32(t):
 SHAPES = [(1, 2, 256, 64), (1, 1, 32, 128), (2, 3, 160, 96), (1, 2, 544, 128), (1, 1, 1024, 96)]
 
 
+@pytest.mark.parametrize("one_pass", [True, False])
 @pytest.mark.parametrize("b,h,n,d", SHAPES)
-def test_dense_attention_lse_and_mass(ops, b, h, n, d):
+def test_dense_attention_lse_and_mass(ops, b, h, n, d, one_pass):
+    """Both block-mass paths: one pass (per-block log-sum-exps recorded by the
+    attention kernel) and two passes (Q K^T recomputed with the final lse)."""
     qb, kb, vb = rand_qkv_bits(b, h, n, d, seed=n + d)
     q, k, v = to_dev(qb), to_dev(kb), to_dev(vb)
-    o, lse, mass = ops.full_attn_mass(q, k, v, with_mass=True)
+    o, lse, mass = ops.full_attn_mass(q, k, v, with_mass=True, one_pass=one_pass)
     torch.cuda.synchronize()
     assert ops.device_status() == 0
     o, lse, mass = dev_f32(o), lse.cpu().numpy(), mass.cpu().numpy()
