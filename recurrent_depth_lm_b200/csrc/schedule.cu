@@ -10,10 +10,11 @@
 //   count : popcount of each row's admissible bits (thread per row), block sums
 //           -> workspace
 //   scan  : exclusive scan of the block sums (one CTA), total -> row_offsets[rows]
-//   emit  : block-local exclusive scan + block base -> row_offsets[row]; then one
-//           warp per row writes its set bits in ascending order -> col_idx, each
-//           lane expanding one 32-bit word at its warp-scanned offset (clamped to
-//           capacity).
+//   emit  : the block's bitmask words are staged in shared memory; block-local
+//           exclusive scan + block base -> row_offsets[row]; then every
+//           (row, word) item is expanded by its own thread at the row's offset
+//           plus the popcount of the row's earlier words (ascending order,
+//           clamped to capacity).
 
 #include <cstdint>
 
@@ -23,6 +24,7 @@ namespace wise {
 
 constexpr int kSchedThreads = 256;
 constexpr int kSchedWarps = kSchedThreads / 32;
+constexpr int kMaxSchedWords = 16;   // bitmask words per row: nq <= 512
 
 __device__ __forceinline__ uint32_t admissible_word(const uint32_t* ub, long long row, int W, int w,
                                                     int q) {
@@ -101,40 +103,37 @@ __global__ void __launch_bounds__(kSchedThreads)
                       long long capacity, long long rows, int nq) {
   __shared__ int warp_sums[32];
   __shared__ int row_off[kSchedThreads];
+  __shared__ uint32_t words[kSchedThreads * kMaxSchedWords];
   const int W = (nq + 31) >> 5;
   const long long row0 = (long long)blockIdx.x * kSchedThreads;
-  const long long row = row0 + threadIdx.x;
-  const int c = row < rows ? row_count(ub, row, W, nq) : 0;
+  const int nrows = (rows - row0 < kSchedThreads) ? (int)(rows - row0) : kSchedThreads;
+  // stage this block's admissible bitmask words (coalesced)
+  for (int x = threadIdx.x; x < nrows * W; x += kSchedThreads) {
+    const int rr = x / W, w = x % W;
+    const long long r = row0 + rr;
+    words[rr * W + w] = admissible_word(ub, r, W, w, (int)(r % nq));
+  }
+  __syncthreads();
+  int c = 0;
+  if (threadIdx.x < nrows)
+    for (int w = 0; w < W; ++w) c += __popc(words[threadIdx.x * W + w]);
   int total;
   const int inc = block_inclusive_scan(c, warp_sums, &total);
   const int off = block_base[blockIdx.x] + inc - c;
   row_off[threadIdx.x] = off;
-  if (row < rows) row_offsets[row] = off;
+  if (threadIdx.x < nrows) row_offsets[row0 + threadIdx.x] = off;
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int rr = warp; rr < kSchedThreads; rr += kSchedWarps) {
-    const long long r = row0 + rr;
-    if (r >= rows) break;
-    const int q = (int)(r % nq);
-    long long pos = row_off[rr];
-    for (int w0 = 0; w0 < W; w0 += 32) {
-      const int w = w0 + lane;
-      uint32_t word = w < W ? admissible_word(ub, r, W, w, q) : 0u;
-      const int cnt = __popc(word);
-      int pre = cnt;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, pre, o);
-        if (lane >= o) pre += y;
-      }
-      long long at = pos + pre - cnt;
-      while (word != 0u) {
-        const int b = __ffs(word) - 1;
-        word &= word - 1u;
-        if (at < capacity) col_idx[at] = w * 32 + b;
-        ++at;
-      }
-      pos += __shfl_sync(0xffffffffu, pre, 31);
+  // expand every (row, word) item independently: its bits go after the row's earlier words
+  for (int x = threadIdx.x; x < nrows * W; x += kSchedThreads) {
+    const int rr = x / W, w = x % W;
+    uint32_t word = words[rr * W + w];
+    long long at = row_off[rr];
+    for (int w2 = 0; w2 < w; ++w2) at += __popc(words[rr * W + w2]);
+    while (word != 0u) {
+      const int b = __ffs(word) - 1;
+      word &= word - 1u;
+      if (at < capacity) col_idx[at] = w * 32 + b;
+      ++at;
     }
   }
 }
