@@ -533,7 +533,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--e2e-reps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
-    ap.add_argument("--cpu-heads", type=int, default=2)
+    ap.add_argument("--cpu-heads", type=int, default=16)
     ap.add_argument("--no-clocks", dest="clocks", action="store_false")
     args = ap.parse_args(argv)
     if args.warmup < 3:

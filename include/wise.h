@@ -198,6 +198,16 @@ int wise_sparse_attn(const void* q, const void* k, const void* v, void* o,
                      float* lse, wise_shape_t shape, void* stream);
 
 /*
+ * Diagnostic (no counterpart in the WISE paper): exercise the bounded pipeline
+ * wait of the kernels.  Launches one warp that waits, with the same bounded wait
+ * the attention kernels use, on an mbarrier phase nothing completes; after
+ * limit_ns nanoseconds the wait gives up, sets WISE_STATUS_TIMEOUT in the device
+ * status word and the kernel returns (the context stays usable).  limit_ns must
+ * be in (0, 10 s].  Errors: WISE_ERR_ARG, WISE_ERR_CUDA.
+ */
+int wise_diag_wait_timeout(uint64_t limit_ns, void* stream);
+
+/*
  * Read (and optionally clear) the device status word of the current device.
  * Synchronises the device.  *status_out receives WISE_STATUS_* bits.
  */

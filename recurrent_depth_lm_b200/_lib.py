@@ -58,6 +58,7 @@ _SIGNATURES = {
                                                   ctypes.POINTER(ctypes.c_int64), WiseShape, _vp]),
     "wise_sparse_attn": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int64, _vp,
                                         WiseShape, _vp]),
+    "wise_diag_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, _vp]),
     "wise_device_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]),
     "wise_last_error": (ctypes.c_char_p, []),
     "wise_version": (ctypes.c_char_p, []),

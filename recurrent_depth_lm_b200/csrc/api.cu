@@ -168,6 +168,13 @@ namespace wise {
 int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
 int record_ok() { return ok(); }
 int validate_shape(const wise_shape_t& s) { return check_shape(s); }
+int status_word(unsigned int** out) {
+  DeviceInfo* di = nullptr;
+  const int rc = device_info(&di);
+  if (rc) return rc;
+  *out = di->status;
+  return WISE_OK;
+}
 }  // namespace wise
 
 extern "C" {

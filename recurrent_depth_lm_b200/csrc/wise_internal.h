@@ -48,5 +48,7 @@ cudaError_t launch_build_schedule(const uint32_t* union_bits, int32_t* row_offse
 int record_error(int code, const char* msg);
 int record_ok();
 int validate_shape(const wise_shape_t& s);
+// Device address of the current device's status word.
+int status_word(unsigned int** out);
 
 }  // namespace wise

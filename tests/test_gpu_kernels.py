@@ -263,3 +263,24 @@ def test_build_schedule_capacity_error(ops):
     assert e.value.code == -4
     with pytest.raises(WiseError):
         ops.build_schedule(bits, col_idx=small, exact_nnz=False)
+
+
+def test_bounded_wait_times_out_and_context_survives(ops):
+    """Failure detection without a GPU fault: a pipeline wait that nothing completes
+    gives up after its limit, records WISE_STATUS_TIMEOUT, and the context stays
+    usable (an attention call right after still matches the oracle)."""
+    import time
+    from recurrent_depth_lm_b200._lib import WISE_STATUS_TIMEOUT, check, lib
+    ops.device_status(clear=True)
+    t0 = time.perf_counter()
+    check(lib.wise_diag_wait_timeout(50_000_000, torch.cuda.current_stream().cuda_stream),
+          "wise_diag_wait_timeout")
+    st = ops.device_status(clear=True)
+    elapsed = time.perf_counter() - t0
+    assert st & WISE_STATUS_TIMEOUT
+    assert 0.04 <= elapsed < 5.0
+    assert ops.device_status() == 0
+    qb, kb, vb = rand_qkv_bits(1, 1, 128, 64, seed=21)
+    o, _, _ = ops.full_attn_mass(to_dev(qb), to_dev(kb), to_dev(vb))
+    o_ref, _ = O.causal_attention(*(bf16_bits_to_f64(x[0, 0]) for x in (qb, kb, vb)))
+    compare_o(dev_f32(o)[0, 0], o_ref)
