@@ -137,17 +137,16 @@ int launch_attn(int mode, const void* q, const void* k, const void* v, void* o,
   int rc = device_info(&di);
   if (rc) return rc;
   const int BH = s.batch * s.heads;
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
   if ((rc = make_tmap(&tq, q, s.head_dim, s.seqlen, BH, 128))) return rc;
   if ((rc = make_tmap(&tk, k, s.head_dim, s.seqlen, BH, 32))) return rc;
   if (mode != wise::kModeMass) {
     if ((rc = make_tmap(&tv, v, s.head_dim, s.seqlen, BH, 32))) return rc;
-    if ((rc = make_tmap(&to, o, s.head_dim, s.seqlen, BH, 128))) return rc;
   } else {
     tv = tk;
-    to = tq;
   }
   wise::AttnParams p = p0;
+  p.o = o;
   p.BH = BH;
   p.n = s.seqlen;
   p.nq = s.seqlen / 32;
@@ -155,9 +154,13 @@ int launch_attn(int mode, const void* q, const void* k, const void* v, void* o,
   p.scale_log2 = softmax_scale(s) * 1.4426950408889634f;
   p.status = di->status;
   const int grid = p.num_tiles < di->sms ? p.num_tiles : di->sms;
-  cudaError_t e = wise::launch_attention(mode, s.head_dim, tq, tk, tv, to, p, grid,
-                                         static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  const char* why = nullptr;
+  cudaError_t e = wise::launch_attention(mode, s.head_dim, tq, tk, tv, p, grid,
+                                         static_cast<cudaStream_t>(stream), &why);
+  if (e != cudaSuccess) {
+    if (why) return fail(WISE_ERR_CUDA, "attention launch: %s", why);
+    return cuda_fail(e, "attention launch");
+  }
   return WISE_OK;
 }
 

@@ -3,7 +3,7 @@
 // One persistent, warp-specialised kernel template covers three modes:
 //   kDense  : exploration-step causal attention (all admissible key blocks),
 //   kSparse : late-step attention over a CSR key-block schedule,
-//   kMass   : the block-mass pass of an exploration window step.
+//   kMass   : the block-mass pass of an exploration window step (two-pass path).
 //
 // Semantics follow Wan & Chen, "Attention Routing Stabilizes Early:
 // Working-Set Inference for Recurrent-Depth Language Models": section 3
@@ -13,19 +13,29 @@
 // section 7.4 (absent blocks are skipped; scoring, causal mask, online
 // softmax and value aggregation are fused).
 //
-// Tiling.  A CTA tile is 128 query rows = 4 query blocks of 32 (one TMEM lane
-// slice of 32 rows per softmax warp, i.e. one query block per warp).  Each
-// iteration gathers up to 4 key blocks (128 keys) with one 32-row TMA box per
-// block and panel, so the tile's key list may be any ascending set of blocks.
-// A slot's "owner mask" says which of the tile's 4 query blocks may see it;
-// rows of other query blocks get probability 0 for it.
+// Two query tiles in flight ("ping-pong").  A CTA keeps two tile slots
+// X = 0, 1.  Each slot holds a 128-row query tile (4 query blocks of 32 rows),
+// its own S region and O accumulator in tensor memory, and its own softmax
+// warpgroup, which owns whole 128-key rows.  Per slot the work is a chain
+//   QK_X(j) -> softmax_X(j) -> PV_X(j) -> QK_X(j+1)
+// (S_X is reused, and P_X lives in S_X), so one slot alone would leave the
+// tensor core idle during its softmax.  The single MMA thread therefore
+// alternates between the slots -- PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1), ... --
+// and the tensor core runs one slot's PV and QK while the other slot's softmax
+// runs.  A slot that finishes its tile takes the CTA's next tile while the other
+// slot keeps the tensor core busy; its output is written from registers, so the
+// next query tile can be loaded as soon as the last QK of the previous one is done.
+//
+// Each iteration gathers up to 4 key blocks (128 keys) with one 32-row TMA box
+// per block and panel, so a tile's key list may be any ascending set of blocks.
+// A slot's "owner mask" says which of the tile's 4 query blocks may see a key
+// block; rows of other query blocks get probability 0 for it.
 //
 // Shared memory (128-byte swizzle, 1024-byte aligned panels of 64 columns):
-//   Q tile [128 x d], K and V stage rings [128 keys x d], P [128 x 128] bf16.
-// Tensor memory: S double buffer (2 x 128 fp32 columns) + one O accumulator
-// per softmax half (2 x 128 columns).  Each half writes its P (bf16, two per
-// column) over the first 32 columns of its own 64-column part of the S buffer
-// it just read, and the PV MMA reads P from there (A operand in TMEM).
+//   Q tiles [2][128 x d], K stage ring and V stage ring [128 keys x d] (both
+//   filled in the CTA's global order of work entries), entry rings, masks.
+// Tensor memory: S_X = columns [128 X, 128 X + 128); O_X = [256 + 128 X, +d).
+// P_X (bf16, two per column) is written over the first 64 columns of S_X.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -38,48 +48,62 @@ namespace wise {
 
 constexpr int kBM = 128;        // query rows per tile
 constexpr int kSlots = 4;       // key blocks per iteration
-constexpr int kThreads = 352;   // 11 warps
+constexpr int kThreads = 384;   // 3 warpgroups
 constexpr int kPanelRowBytes = 128;                // 64 bf16 per swizzled row
 constexpr int kPanelBytes = kBM * kPanelRowBytes;  // one 128-row panel = 16 KB
 constexpr int kMaxWords = 16;   // schedule bitmask words per query block (nq <= 512)
-constexpr int kInfoRing = 8;    // iterations of slot info in flight
-constexpr int kSoftmaxThreads = 256;  // two halves of 4 warps
+constexpr int kRing = 4;        // work entries in flight per tile slot
+
+// Register split (setmaxnreg): the launch gives every thread kLaunchRegs; the
+// control warpgroup (TMA producers, MMA issuer) drops to kCtlRegs and the two
+// softmax warpgroups rise to kSoftRegs.  The sum must not exceed the launch's.
+constexpr int kLaunchRegs = 168;
+constexpr int kCtlRegs = 72;
+constexpr int kSoftRegs = 216;
+static_assert(128 * kCtlRegs + 256 * kSoftRegs <= kLaunchRegs * kThreads, "register split");
+static_assert(kLaunchRegs * kThreads <= 65536, "register file");
+
+enum : int { kWork = 0, kEnd = 1 };
+enum : int { kFirst = 1, kLast = 2 };
+
+// One work entry of a tile slot: one iteration of up to 4 key blocks, or the
+// end marker of the slot.  Written by the Q/K producer, read by the V
+// producer, the MMA issuer and the slot's softmax warpgroup.
+struct Entry {
+  int kind;
+  int flags;   // kFirst / kLast of the slot's current tile
+  int ns;      // key blocks used (1..4)
+  int bh;
+  int Qt;
+  int stage;   // index among the CTA's work entries: K ring = stage % NK, V ring = stage % NV
+  int pad0, pad1;
+  int kb[kSlots];
+  int own[kSlots];
+};
+static_assert(sizeof(Entry) == 64, "entry layout");
 
 template <int D, int MODE>
 struct Cfg {
   static constexpr int kPanels = (D + 63) / 64;
   static constexpr bool kAttn = MODE != kModeMass;
   static constexpr int kTileBytes = kPanels * kPanelBytes;  // Q tile, one K or V stage
-  // K ring (freed when QK finishes) and V ring (freed when PV finishes).
-  static constexpr int kKStages = kAttn ? (D <= 64 ? 4 : 3) : 4;
+  static constexpr int kKStages = kAttn ? (D <= 64 ? 4 : 3) : (D <= 64 ? 6 : 4);
   static constexpr int kVStages = kAttn ? (D <= 64 ? 4 : 2) : 0;
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kTileBytes;
-  static constexpr int kOffV = kOffK + kKStages * kTileBytes;
-  static constexpr int kOffX = kOffV + kVStages * kTileBytes;   // epilogue (m, l) exchange
-  static constexpr int kOffInfo = kOffX + (kAttn ? 2 * kBM * 8 : 0);
-  static constexpr int kInfoBytes = 64;
-  static constexpr int kOffMask = kOffInfo + kInfoRing * kInfoBytes;
-  static constexpr int kOffBar = kOffMask + 4 * kMaxWords * 4;
   static constexpr int kVRing = kVStages > 0 ? kVStages : 1;  // barrier slots (mass mode: unused)
-  // q_full, q_empty, k_full[K], k_empty[K], v_full[V], v_empty[V], info_full[I], info_empty[I],
-  // s_full[2], s_free[2], p_full[2 halves][2 S buffers], o_done[2], merge, o_staged, final
-  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVRing + 2 * kInfoRing + 14;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + 2 * kTileBytes;
+  static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+  static constexpr int kOffEnt = kOffV + kVStages * kTileBytes;
+  static constexpr int kOffMask = kOffEnt + 2 * kRing * (int)sizeof(Entry);
+  static constexpr int kOffBar = kOffMask + 2 * 4 * kMaxWords * 4;
+  // q_full[2], q_empty[2], k_full[K], k_empty[K], v_full[V], v_empty[V], e_full[2][R],
+  // e_empty[2][R], s_full[2], s_free[2], p_full[2], o_done[2], o_free[2], final
+  static constexpr int kNumBars = 4 + 2 * kKStages + 2 * kVRing + 4 * kRing + 11;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
   static constexpr uint32_t kTmemCols = kAttn ? 512 : 256;
-  static constexpr uint32_t kOCol = 256;   // O of half h at kOCol + 128 * h
+  static constexpr uint32_t kOCol = 256;   // O of slot X at kOCol + 128 * X
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(kInfoRing >= kKStages + 1, "info slot reuse needs QK of its iteration done");
-};
-
-struct StageInfo {
-  int nslots;
-  int last;
-  int bh;
-  int pad;
-  int kb[kSlots];
-  int own[kSlots];
 };
 
 // ---------------------------------------------------------------- key-block lists
@@ -180,6 +204,11 @@ __device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
+// kb[s] of a 4-entry register array for a runtime s, without local memory.
+__device__ __forceinline__ int pick4(const int (&v)[4], int s) {
+  return s == 0 ? v[0] : s == 1 ? v[1] : s == 2 ? v[2] : v[3];
+}
+
 // Warp-uniform bounded wait: every lane polls, the warp agrees on the outcome.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           unsigned int* status) {
@@ -189,32 +218,45 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return ok;
 }
 
+// The CTA's k-th tile: waves of gridDim.x tiles, every other wave in reverse CTA
+// order, over tiles sorted heaviest first (largest Qt, most key blocks).
+__device__ __forceinline__ int cta_tile(int k, int num_tiles) {
+  const int G = gridDim.x;
+  const int t = k * G + ((k & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+  return t < num_tiles ? t : -1;
+}
+
 __device__ __forceinline__ void decode_tile(int tile, int BH, int ntq, int& bh, int& Qt) {
-  // heaviest tiles (largest Qt, most key blocks) first
   Qt = ntq - 1 - tile / BH;
   bh = tile % BH;
 }
 
+__device__ __forceinline__ void st_global_v4(void* ptr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(ptr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
 // ---------------------------------------------------------------- the kernel
 //
-// Warp roles (352 threads): warp 0 = Q/K TMA producer and slot-list writer;
-// warp 1 = TMEM allocator + single-thread MMA issuer; warp 2 = V TMA producer;
-// warps 3..10 = softmax in two halves.  Half h (warps 3+4h .. 6+4h) owns key
-// slots 2h and 2h+1 of every iteration (S columns 64h..64h+63)
-// and keeps its own online-softmax state (m, l) and its own O accumulator in
-// TMEM; the two partial results of a row are merged once, in the epilogue:
-//   O = (2^(m_a-m) O_a + 2^(m_b-m) O_b) / (2^(m_a-m) l_a + 2^(m_b-m) l_b).
-// Warp w reads TMEM lane quarter w % 4 (rows 32*(w%4) .. +31), i.e. one query
-// block of the tile per warp.
+// Warp roles (384 threads, 3 warpgroups):
+//   warpgroup 0: warp 0 = Q/K TMA producer and entry writer (whole warp: sparse
+//     masks), warp 1 = TMEM allocator + single-thread MMA issuer, warp 2 = V TMA
+//     producer, warp 3 = idle;
+//   warpgroup 1 (warps 4..7) = softmax of slot 0, warpgroup 2 (warps 8..11) =
+//     softmax of slot 1.  Warp w reads TMEM lane quarter w % 4 (rows
+//     32*(w%4) .. +31), i.e. one query block of its slot's tile; thread = row.
+// Every party walks the two slot rings in the same order: alternate slots,
+// skipping a slot once its end entry has been read.
 
 template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                const AttnParams p) {
+                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using C = Cfg<D, MODE>;
   constexpr int NK = C::kKStages;
-  constexpr int NV = C::kVRing;  // mass mode has no V ring; its barrier slots stay unused
+  constexpr int NV = C::kVRing;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
 
@@ -224,41 +266,51 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sQ = smem_u32(smem + C::kOffQ);
   const uint32_t sK = smem_u32(smem + C::kOffK);
   const uint32_t sV = smem_u32(smem + C::kOffV);
-  StageInfo* info = (StageInfo*)(smem + C::kOffInfo);
-  uint32_t* tile_mask = (uint32_t*)(smem + C::kOffMask);
+  Entry* ents = (Entry*)(smem + C::kOffEnt);               // [2][kRing]
+  uint32_t* masks = (uint32_t*)(smem + C::kOffMask);       // [2][4][kMaxWords]
   const uint32_t bar0 = smem_u32(smem + C::kOffBar);
-  const uint32_t bar_q_full = bar0;
-  const uint32_t bar_q_empty = bar0 + 8;
-  const uint32_t barK = bar0 + 16;
+  auto bar_q_full = [&](int x) { return bar0 + 8 * x; };
+  auto bar_q_empty = [&](int x) { return bar0 + 16 + 8 * x; };
+  const uint32_t barK = bar0 + 32;
   auto bar_k_full = [&](int s) { return barK + 8 * s; };
   auto bar_k_empty = [&](int s) { return barK + 8 * NK + 8 * s; };
   const uint32_t barV = barK + 16 * NK;
   auto bar_v_full = [&](int s) { return barV + 8 * s; };
   auto bar_v_empty = [&](int s) { return barV + 8 * NV + 8 * s; };
-  const uint32_t barI = barV + 16 * NV;
-  auto bar_i_full = [&](int s) { return barI + 8 * s; };
-  auto bar_i_empty = [&](int s) { return barI + 8 * kInfoRing + 8 * s; };
-  const uint32_t barS = barI + 16 * kInfoRing;
-  auto bar_s_full = [&](int b) { return barS + 8 * b; };
-  auto bar_s_free = [&](int b) { return barS + 16 + 8 * b; };
-  // one p_full per (half, S buffer): the softmax may run an iteration ahead of the
-  // MMA issuer, so a single barrier per half could complete two phases unobserved
-  auto bar_p_full = [&](int h, int b) { return barS + 32 + 16 * h + 8 * b; };
-  // one o_done per S buffer: arrives when both halves' PV of an iteration using that
-  // buffer has completed (phase index = iteration >> 1)
-  auto bar_o_done = [&](int b) { return barS + 64 + 8 * b; };
-  const uint32_t bar_merge = barS + 80;
-  const uint32_t bar_o_staged = barS + 88;
-  const uint32_t bar_final = barS + 96;
+  const uint32_t barE = barV + 16 * NV;
+  auto bar_e_full = [&](int x, int k) { return barE + 8 * (x * kRing + k); };
+  auto bar_e_empty = [&](int x, int k) { return barE + 16 * kRing + 8 * (x * kRing + k); };
+  const uint32_t barS = barE + 32 * kRing;
+  auto bar_s_full = [&](int x) { return barS + 8 * x; };
+  auto bar_s_free = [&](int x) { return barS + 16 + 8 * x; };   // mass mode: S read
+  auto bar_p_full = [&](int x) { return barS + 32 + 8 * x; };   // P_X written
+  auto bar_o_done = [&](int x) { return barS + 48 + 8 * x; };   // PV_X complete
+  auto bar_o_free = [&](int x) { return barS + 64 + 8 * x; };   // O_X read by the epilogue
+  const uint32_t bar_final = barS + 80;
   volatile int* abort_flag = (volatile int*)(smem + C::kOffMisc);
   uint32_t* tmem_slot = (uint32_t*)(smem + C::kOffMisc + 4);
+  // abort flag of the drain waits at exit, which must not give up early
+  volatile int* drain_flag = (volatile int*)(smem + C::kOffMisc + 8);
 
   const int ntq = (p.nq + 3) / 4;
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    mbar_init(bar_q_full, 1);
-    mbar_init(bar_q_empty, 1);
+    *drain_flag = 0;
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar_q_full(x), 1);
+      mbar_init(bar_q_empty(x), 1);
+      for (int k = 0; k < kRing; ++k) {
+        mbar_init(bar_e_full(x, k), 1);
+        // read by the slot's 128 softmax threads, the MMA issuer and (attention) the V producer
+        mbar_init(bar_e_empty(x, k), 128 + 1 + (C::kAttn ? 1 : 0));
+      }
+      mbar_init(bar_s_full(x), 1);
+      mbar_init(bar_s_free(x), 128);
+      mbar_init(bar_p_full(x), 128);
+      mbar_init(bar_o_done(x), 1);
+      mbar_init(bar_o_free(x), 128);
+    }
     for (int s = 0; s < NK; ++s) {
       mbar_init(bar_k_full(s), 1);
       mbar_init(bar_k_empty(s), 1);
@@ -267,20 +319,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_v_full(s), 1);
       mbar_init(bar_v_empty(s), 1);
     }
-    for (int s = 0; s < kInfoRing; ++s) {
-      mbar_init(bar_i_full(s), 1);
-      // read by the 256 softmax threads and, in attention modes, the V producer
-      mbar_init(bar_i_empty(s), kSoftmaxThreads + (C::kAttn ? 1 : 0));
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_s_full(b), 1);
-      mbar_init(bar_s_free(b), kSoftmaxThreads);
-      mbar_init(bar_p_full(0, b), kSoftmaxThreads / 2);
-      mbar_init(bar_p_full(1, b), kSoftmaxThreads / 2);
-      mbar_init(bar_o_done(b), 1);
-    }
-    mbar_init(bar_merge, kSoftmaxThreads);
-    mbar_init(bar_o_staged, kSoftmaxThreads);
     mbar_init(bar_final, 1);
     fence_mbar_init();
   }
@@ -293,502 +331,542 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // Each setmaxnreg sits at the head of its warpgroup's branch, so that the code of
+  // every role is dominated by the register limit that applies to it.
+  if (warp < 4) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtlRegs));
   if (warp == 0) {
-    // ======================================================= Q / K producer, slot lists
+    // ======================================================= Q / K producer, entry writer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
     }
-    uint32_t it = 0;
-    int tl = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tl) {
-      int bh, Qt;
-      decode_tile(tile, p.BH, ntq, bh, Qt);
-      if (MODE == kModeSparse) build_tile_masks(tile_mask, p, bh, Qt, lane);
-      if (lane == 0) {
-        if (tl > 0 && !mbar_wait(bar_q_empty, (tl - 1) & 1, abort_flag, p.status)) ok = false;
-        if (ok) {
-          mbar_arrive_expect_tx(bar_q_full, C::kTileBytes);
+    struct Slot {
+      DenseList dl;
+      MaskList ml;
+      int bh, qt, rc;
+      uint32_t tq;          // tiles started (q_empty phases)
+      bool active, ended, first;
+    };
+    Slot sa{}, sb{};
+    uint32_t g = 0;         // work entries written (K/V stage index)
+    int next_k = 0;
+    // One entry (work or end) for slot X; false on abort.
+    auto step = [&](Slot& S, const int X) -> bool {
+      const int k = S.rc % kRing;
+      if (S.rc >= kRing &&
+          !warp_wait(bar_e_empty(X, k), ((S.rc / kRing) - 1) & 1, abort_flag, p.status))
+        return false;
+      Entry& e = ents[X * kRing + k];
+      if (!S.active) {
+        const int tile = cta_tile(next_k++, p.num_tiles);
+        if (tile < 0) {
+          if (lane == 0) {
+            e.kind = kEnd;
+            mbar_arrive(bar_e_full(X, k));
+          }
+          ++S.rc;
+          S.ended = true;
+          return true;
+        }
+        decode_tile(tile, p.BH, ntq, S.bh, S.qt);
+        if (MODE == kModeSparse) {
+          uint32_t* msk = masks + X * 4 * kMaxWords;
+          build_tile_masks(msk, p, S.bh, S.qt, lane);
+          S.ml.init(msk, (p.nq + 31) / 32);
+        } else {
+          S.dl.init(S.qt, p.nq);
+        }
+        // the slot's previous tile must have finished its QK MMAs before Q_X is overwritten
+        if (S.tq >= 1 && !warp_wait(bar_q_empty(X), (S.tq - 1) & 1, abort_flag, p.status))
+          return false;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_q_full(X), C::kTileBytes);
           for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_3d(sQ + pn * kPanelBytes, &tmQ, bar_q_full, pn * 64, Qt * kBM, bh);
+            tma_load_3d(sQ + X * C::kTileBytes + pn * kPanelBytes, &tmQ, bar_q_full(X), pn * 64,
+                        S.qt * kBM, S.bh);
         }
-        DenseList dl;
-        MaskList ml;
-        if (MODE == kModeSparse)
-          ml.init(tile_mask, (p.nq + 31) / 32);
-        else
-          dl.init(Qt, p.nq);
-        bool first = true;
-        while (ok) {
-          int kbv[kSlots], ownv[kSlots];
-          int n = 0;
-          int kb, own;
-          while (n < kSlots && (MODE == kModeSparse ? ml.pop(kb, own) : dl.pop(kb, own))) {
-            kbv[n] = kb;
-            ownv[n] = own;
-            ++n;
-          }
-          if (n == 0) {
-            if (!first) break;  // unreachable: `last` was set on the previous group
-            kbv[0] = 0;         // empty tile: one fully masked slot keeps the pipeline uniform
-            ownv[0] = 0;
-            n = 1;
-          }
-          const bool last = (MODE == kModeSparse) ? ml.empty() : dl.empty();
-          const int is = it % kInfoRing;
-          if (it >= (uint32_t)kInfoRing &&
-              !mbar_wait(bar_i_empty(is), ((it / kInfoRing) - 1) & 1, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          StageInfo& si = info[is];
-          si.nslots = n;
-          si.last = last ? 1 : 0;
-          si.bh = bh;
-          for (int s = 0; s < kSlots; ++s) {
-            si.kb[s] = s < n ? kbv[s] : 0;
-            si.own[s] = s < n ? ownv[s] : 0;
-          }
-          mbar_arrive(bar_i_full(is));
-          const int ks = it % NK;
-          if (it >= (uint32_t)NK &&
-              !mbar_wait(bar_k_empty(ks), ((it / NK) - 1) & 1, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar_k_full(ks), (uint32_t)n * 32 * kPanelRowBytes * C::kPanels);
-          const uint32_t kbase = sK + ks * C::kTileBytes;
-          for (int s = 0; s < n; ++s)
-            for (int pn = 0; pn < C::kPanels; ++pn)
-              tma_load_3d(kbase + pn * kPanelBytes + s * 32 * kPanelRowBytes, &tmK, bar_k_full(ks),
-                          pn * 64, kbv[s] * 32, bh);
-          ++it;
-          first = false;
-          if (last) break;
+        ++S.tq;
+        S.active = true;
+        S.first = true;
+      }
+      int kbv[kSlots], ownv[kSlots];
+      int n = 0;
+      {
+        int kb, own;
+        while (n < kSlots && (MODE == kModeSparse ? S.ml.pop(kb, own) : S.dl.pop(kb, own))) {
+          kbv[n] = kb;
+          ownv[n] = own;
+          ++n;
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      it = __shfl_sync(0xffffffffu, it, 0);
-    }
-    if (lane == 0) {  // let the last K loads land before the CTA can exit
-      const uint32_t from = it > (uint32_t)NK ? it - NK : 0u;
-      for (uint32_t j = from; j < it; ++j) {
-        volatile int dummy = 0;
-        mbar_wait(bar_k_full(j % NK), (j / NK) & 1, &dummy, p.status);
+      if (n == 0) {  // empty tile: one fully masked key block keeps the pipeline uniform
+        kbv[0] = 0;
+        ownv[0] = 0;
+        n = 1;
       }
+      const bool last = (MODE == kModeSparse) ? S.ml.empty() : S.dl.empty();
+      const int ks = g % NK;
+      if (g >= (uint32_t)NK &&
+          !warp_wait(bar_k_empty(ks), ((g / NK) - 1) & 1, abort_flag, p.status))
+        return false;
+      if (lane == 0) {
+        e.kind = kWork;
+        e.flags = (S.first ? kFirst : 0) | (last ? kLast : 0);
+        e.ns = n;
+        e.bh = S.bh;
+        e.Qt = S.qt;
+        e.stage = (int)g;
+        for (int s = 0; s < kSlots; ++s) {
+          e.kb[s] = s < n ? kbv[s] : 0;
+          e.own[s] = s < n ? ownv[s] : 0;
+        }
+        mbar_arrive(bar_e_full(X, k));
+        mbar_arrive_expect_tx(bar_k_full(ks), (uint32_t)n * 32 * kPanelRowBytes * C::kPanels);
+        const uint32_t kbase = sK + ks * C::kTileBytes;
+#pragma unroll 1
+        for (int s = 0; s < n; ++s) {
+          const int kb = pick4(kbv, s);
+#pragma unroll
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_load_3d(kbase + pn * kPanelBytes + s * 32 * kPanelRowBytes, &tmK, bar_k_full(ks),
+                        pn * 64, kb * 32, S.bh);
+        }
+      }
+      ++S.rc;
+      ++g;
+      S.first = false;
+      if (last) S.active = false;
+      return true;
+    };
+    // Alternate slots, skipping a slot that has ended.  One call site: the slot's
+    // state is selected into S and written back (keeps the code compact).
+    bool ok = true;
+    for (int X = 0; ok && !(sa.ended && sb.ended); X ^= 1) {
+      if (X == 0 ? sa.ended : sb.ended) continue;
+      Slot S = X == 0 ? sa : sb;
+      ok = step(S, X);
+      if (X == 0) sa = S; else sb = S;
     }
+    if (lane == 0) {  // let the last K and Q loads land before the CTA can exit
+      const uint32_t from = g > (uint32_t)NK ? g - NK : 0u;
+      for (uint32_t j = from; j < g; ++j) {
+        mbar_wait(bar_k_full(j % NK), (j / NK) & 1, drain_flag, p.status);
+      }
+      if (sa.tq >= 1) mbar_wait(bar_q_full(0), (sa.tq - 1) & 1, drain_flag, p.status);
+      if (sb.tq >= 1) mbar_wait(bar_q_full(1), (sb.tq - 1) & 1, drain_flag, p.status);
+    }
+    __syncwarp();
   } else if (warp == 2) {
     // ======================================================= V producer (attention modes)
     if (C::kAttn && lane == 0) {
       tma_prefetch_desc(&tmV);
-      uint32_t it = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-        while (true) {
-          const int is = it % kInfoRing;
-          if (!mbar_wait(bar_i_full(is), (it / kInfoRing) & 1, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          const int n = info[is].nslots;
-          const int last = info[is].last;
-          const int bh = info[is].bh;
-          int kbv[kSlots];
+      struct Slot {
+        int rc;
+        bool ended;
+      };
+      Slot sa{}, sb{};
+      uint32_t issued = 0;
+      auto step = [&](Slot& S, const int X) -> bool {
+        const int k = S.rc % kRing;
+        if (!mbar_wait(bar_e_full(X, k), (S.rc / kRing) & 1, abort_flag, p.status)) return false;
+        const Entry& e = ents[X * kRing + k];
+        const int kind = e.kind;
+        const int n = e.ns;
+        const int bh = e.bh;
+        const uint32_t g = (uint32_t)e.stage;
+        int kbv[kSlots];
 #pragma unroll
-          for (int s = 0; s < kSlots; ++s) kbv[s] = info[is].kb[s];
-          mbar_arrive(bar_i_empty(is));
-          const int vs = it % NV;
-          if (it >= (uint32_t)NV &&
-              !mbar_wait(bar_v_empty(vs), ((it / NV) - 1) & 1, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar_v_full(vs), (uint32_t)n * 32 * kPanelRowBytes * C::kPanels);
-          const uint32_t vbase = sV + vs * C::kTileBytes;
-          for (int s = 0; s < n; ++s)
-            for (int pn = 0; pn < C::kPanels; ++pn)
-              tma_load_3d(vbase + pn * kPanelBytes + s * 32 * kPanelRowBytes, &tmV, bar_v_full(vs),
-                          pn * 64, kbv[s] * 32, bh);
-          ++it;
-          if (last) break;
+        for (int s = 0; s < kSlots; ++s) kbv[s] = e.kb[s];
+        mbar_arrive(bar_e_empty(X, k));
+        ++S.rc;
+        if (kind == kEnd) {
+          S.ended = true;
+          return true;
         }
+        const int vs = g % NV;
+        if (g >= (uint32_t)NV &&
+            !mbar_wait(bar_v_empty(vs), ((g / NV) - 1) & 1, abort_flag, p.status))
+          return false;
+        mbar_arrive_expect_tx(bar_v_full(vs), (uint32_t)n * 32 * kPanelRowBytes * C::kPanels);
+        const uint32_t vbase = sV + vs * C::kTileBytes;
+#pragma unroll 1
+        for (int s = 0; s < n; ++s) {
+          const int kb = pick4(kbv, s);
+#pragma unroll
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_load_3d(vbase + pn * kPanelBytes + s * 32 * kPanelRowBytes, &tmV, bar_v_full(vs),
+                        pn * 64, kb * 32, bh);
+        }
+        issued = g + 1;
+        return true;
+      };
+      bool ok = true;
+      for (int X = 0; ok && !(sa.ended && sb.ended); X ^= 1) {
+        if (X == 0 ? sa.ended : sb.ended) continue;
+        Slot S = X == 0 ? sa : sb;
+        ok = step(S, X);
+        if (X == 0) sa = S; else sb = S;
       }
-      const uint32_t from = it > (uint32_t)NV ? it - NV : 0u;
-      for (uint32_t j = from; j < it; ++j) {
-        volatile int dummy = 0;
-        mbar_wait(bar_v_full(j % NV), (j / NV) & 1, &dummy, p.status);
+      const uint32_t from = issued > (uint32_t)NV ? issued - NV : 0u;
+      for (uint32_t j = from; j < issued; ++j) {
+        mbar_wait(bar_v_full(j % NV), (j / NV) & 1, drain_flag, p.status);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ======================================================= MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the issuer (converged, so its descriptor arithmetic stays
+    // warp-uniform); one elected lane issues each MMA, commit and arrival.
+    {
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);
-      uint32_t it = 0;
-      int tl = 0;
-      bool ok = true;
+      struct Slot {
+        int rc;
+        bool ended;
+        bool pend;          // a work entry whose PV is not issued yet
+        bool pend_first;
+        int pend_ns, pend_stage;
+        uint32_t pvc;       // PVs issued (p_full / o_done phases)
+        uint32_t qkc;       // QKs issued (s_free phases)
+        uint32_t qtiles;    // tiles whose first QK was issued (q_full phases)
+        uint32_t otiles;    // tiles whose first PV was issued (o_free phases)
+      };
+      Slot sa{}, sb{};
       bool issued = false;
-      // S_j = Q K_j^T into S buffer j&1; returns the iteration's slot count and last flag.
-      auto issue_qk = [&](uint32_t j, int& ns, int& last) -> bool {
-        const int ks = j % NK;
-        if (!mbar_wait(bar_k_full(ks), (j / NK) & 1, abort_flag, p.status)) return false;
-        if (j >= 2) {
-          // S buffer j&1 still holds S_{j-2} (mass mode) or P_{j-2} (attention modes)
-          if (!C::kAttn) {
-            if (!mbar_wait(bar_s_free(j & 1), ((j >> 1) - 1) & 1, abort_flag, p.status))
-              return false;
-          } else if (!mbar_wait(bar_o_done(j & 1), ((j >> 1) - 1) & 1, abort_flag, p.status)) {
-            return false;   // PV_{j-2} has read its P out of buffer j&1
-          }
+
+      // O_X (+)= P_X V of the slot's pending entry; P_X is read from TMEM (S_X columns).
+      auto issue_pv = [&](Slot& S, const int X) -> bool {
+        if (!warp_wait(bar_p_full(X), S.pvc & 1, abort_flag, p.status)) return false;
+        if (S.pend_first) {
+          // the first PV of a tile overwrites O_X: the previous tile's epilogue must have read it
+          if (S.otiles >= 1 &&
+              !warp_wait(bar_o_free(X), (S.otiles - 1) & 1, abort_flag, p.status))
+            return false;
+          ++S.otiles;
+        }
+        const uint32_t g = (uint32_t)S.pend_stage;
+        const int vs = g % NV;
+        if (!warp_wait(bar_v_full(vs), (g / NV) & 1, abort_flag, p.status)) return false;
+        tc_fence_after();
+        const uint32_t vbase = sV + vs * C::kTileBytes;
+        const uint32_t p_tmem = tmem_base + X * 128;
+        const uint32_t o_tmem = tmem_base + C::kOCol + X * 128;
+        const int nk = 2 * S.pend_ns;
+        for (int kk = 0; kk < nk; ++kk) {
+          const uint64_t b = smem_desc_sw128(vbase + kk * 16 * kPanelRowBytes, kPanelBytes, 1024);
+          mma_bf16_ts_warp(o_tmem, p_tmem + kk * 8, b, idesc_o, (S.pend_first && kk == 0) ? 0u : 1u);
+        }
+        mma_commit_warp(bar_o_done(X));
+        mma_commit_warp(bar_v_empty(vs));
+        ++S.pvc;
+        S.pend = false;
+        issued = true;
+        return true;
+      };
+
+      // Read slot X's next entry: PV of its previous entry, then QK of this one.
+      auto step = [&](Slot& S, const int X) -> bool {
+        const int k = S.rc % kRing;
+        if (!warp_wait(bar_e_full(X, k), (S.rc / kRing) & 1, abort_flag, p.status)) return false;
+        const Entry& e = ents[X * kRing + k];
+        const int kind = e.kind;
+        const int flags = e.flags;
+        const int ns = e.ns;
+        const int stage = e.stage;
+        __syncwarp();
+        mbar_arrive_warp(bar_e_empty(X, k));
+        ++S.rc;
+        if (C::kAttn && S.pend && !issue_pv(S, X)) return false;
+        if (kind == kEnd) {
+          S.ended = true;
+          return true;
+        }
+        // ---- S_X = Q_X K^T
+        const int ks = stage % NK;
+        if (!warp_wait(bar_k_full(ks), (stage / NK) & 1, abort_flag, p.status)) return false;
+        if (flags & kFirst) {
+          if (!warp_wait(bar_q_full(X), S.qtiles & 1, abort_flag, p.status)) return false;
+          ++S.qtiles;
+        }
+        if (S.qkc >= 1) {
+          // S_X holds the previous P_X (read by the PV just issued) or, in mass mode, the
+          // previous S_X (read by the softmax warps)
+          const bool w = C::kAttn
+                             ? warp_wait(bar_o_done(X), (S.pvc - 1) & 1, abort_flag, p.status)
+                             : warp_wait(bar_s_free(X), (S.qkc - 1) & 1, abort_flag, p.status);
+          if (!w) return false;
         }
         tc_fence_after();
-        ns = info[j % kInfoRing].nslots;
-        last = info[j % kInfoRing].last;
         const uint32_t idesc = idesc_bf16_f32(128, 32 * ns, 0, 0);
-        const uint32_t d_tmem = tmem_base + (j & 1) * 128;
+        const uint32_t d_tmem = tmem_base + X * 128;
+        const uint32_t qbase = sQ + X * C::kTileBytes;
         const uint32_t kbase = sK + ks * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
-          mma_bf16_ss(d_tmem, smem_desc_sw128(sQ + off, 16, 1024),
-                      smem_desc_sw128(kbase + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+          mma_bf16_ss_warp(d_tmem, smem_desc_sw128(qbase + off, 16, 1024),
+                           smem_desc_sw128(kbase + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar_s_full(j & 1));
-        mma_commit(bar_k_empty(ks));
+        mma_commit_warp(bar_s_full(X));
+        mma_commit_warp(bar_k_empty(ks));
+        if (flags & kLast) mma_commit_warp(bar_q_empty(X));  // Q_X may be reloaded
+        ++S.qkc;
         issued = true;
+        if (C::kAttn) {
+          S.pend = true;
+          S.pend_ns = ns;
+          S.pend_stage = stage;
+          S.pend_first = (flags & kFirst) != 0;
+        }
         return true;
       };
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tl) {
-        if (!mbar_wait(bar_q_full, tl & 1, abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        bool started[2] = {false, false};  // has half h's O been written in this tile
-        int ns = 0, last = 1;
-        if (!issue_qk(it, ns, last)) {
-          ok = false;
-          break;
-        }
-        while (true) {
-          int ns_next = 0, last_next = 1;
-          if (!last && !issue_qk(it + 1, ns_next, last_next)) {
-            ok = false;
-            break;
-          }
-          if (C::kAttn) {
-            const int vs = it % NV;
-            if (!mbar_wait(bar_v_full(vs), (it / NV) & 1, abort_flag, p.status)) {
-              ok = false;
-              break;
-            }
-            const uint32_t vbase = sV + vs * C::kTileBytes;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              if (!mbar_wait(bar_p_full(h, it & 1), (it >> 1) & 1, abort_flag, p.status)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              // half h: keys 64h .. 64h+63 of the iteration = 16-key steps 4h .. 4h+3;
-              // its P sits in TMEM columns 64h .. 64h+31 of S buffer it&1 (8 per step)
-              const int kend = min(2 * ns, 4 * h + 4);
-              const uint32_t p_tmem = tmem_base + (it & 1) * 128 + 64 * h;
-              for (int kk = 4 * h; kk < kend; ++kk) {
-                const uint64_t b =
-                    smem_desc_sw128(vbase + kk * 16 * kPanelRowBytes, kPanelBytes, 1024);
-                mma_bf16_ts(tmem_base + C::kOCol + 128 * h, p_tmem + (kk - 4 * h) * 8, b, idesc_o,
-                            (started[h] || kk > 4 * h) ? 1u : 0u);
-              }
-              if (kend > 4 * h) started[h] = true;
-            }
-            if (!ok) break;
-            mma_commit(bar_o_done(it & 1));
-            mma_commit(bar_v_empty(vs));
-          }
-          ++it;
-          if (last) break;
-          ns = ns_next;
-          last = last_next;
-        }
-        if (!ok) break;
-        if (!C::kAttn) mma_commit(bar_q_empty);  // Q is free once this tile's QK MMAs finish
+
+      bool ok = true;
+      for (int X = 0; ok && !(sa.ended && sb.ended); X ^= 1) {
+        if (X == 0 ? sa.ended : sb.ended) continue;
+        Slot S = X == 0 ? sa : sb;
+        ok = step(S, X);
+        if (X == 0) sa = S; else sb = S;
       }
       if (issued) {
-        mma_commit(bar_final);
-        volatile int dummy = 0;
-        mbar_wait(bar_final, 0, &dummy, p.status);
+        mma_commit_warp(bar_final);
+        mbar_wait(bar_final, 0, drain_flag, p.status);
       }
+      __syncwarp();
     }
-    __syncwarp();
+  }
   } else {
-    // ======================================================= softmax / epilogue (warps 3..10)
-    const int half = (warp - 3) >> 2;   // key slots 2*half, 2*half+1
-    const int wg = warp & 3;            // TMEM lane quarter owned by this warp
-    const int r = wg * 32 + lane;       // row within the tile
-    const uint32_t t_row = tmem_base + ((uint32_t)(wg * 32) << 16);
-    const uint32_t o_col = C::kOCol + 128 * half;
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftRegs));
+    // ======================================================= softmax / epilogue of slot X
+    // Thread = row.  Each iteration reads its key blocks from S_X twice (row max,
+    // then exponentials), one 32-column block at a time in a rolled loop: the hot
+    // loop stays small enough for the instruction cache.
+    const int X = (warp - 4) >> 2;
+    const int qw = warp & 3;            // TMEM lane quarter = query block within the tile
+    const uint32_t t_lane = tmem_base + ((uint32_t)(qw * 32) << 16);
+    const uint32_t s_col = X * 128;
+    const uint32_t o_col = C::kOCol + X * 128;
     const float sl2 = p.scale_log2;
-    float* xchg = reinterpret_cast<float*>(smem + C::kOffX);
-    uint32_t it = 0;
-    int tl = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tl) {
-      int bh, Qt;
-      decode_tile(tile, p.BH, ntq, bh, Qt);
-      const int qb = Qt * 4 + wg;      // this warp's query block
-      const int i = qb * 32 + lane;    // query row within the head
-      float m = -INFINITY, l = 0.f;
-      float lse_l2 = 0.f;
-      if (!C::kAttn && i < p.n) lse_l2 = p.lse_in[(long long)bh * p.n + i] * 1.4426950408889634f;
-      bool started = false;   // mirrors the MMA issuer: this half's O written in this tile
-      bool wrote_other = false;
+    int rc = 0;
+    uint32_t cnt = 0;                   // work entries processed (s_full / o_done phases)
+    bool run = true;
+    while (run) {
+      // ---------------- one tile of the slot: its entries, then the epilogue
+      float m = -INFINITY, l = 0.f, lse_l2 = 0.f;
+      int bh = 0, qb = 0, i = 0;
+      bool first = true;
       while (true) {
-        const int is = it % kInfoRing;
-        if (!warp_wait(bar_i_full(is), (it / kInfoRing) & 1, abort_flag, p.status)) {
-          ok = false;
+        const int k = rc % kRing;
+        if (!warp_wait(bar_e_full(X, k), (rc / kRing) & 1, abort_flag, p.status)) {
+          run = false;
           break;
         }
-        const int ns = info[is].nslots;
-        const int last = info[is].last;
-        int kbs[2], vld[2];
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          const int s = 2 * half + x;
-          kbs[x] = info[is].kb[s];
-          vld[x] = (s < ns) && ((info[is].own[s] >> wg) & 1);
+        // The entry stays valid until this warp's arrival on e_empty at the end of
+        // the iteration: key-block indices are read from it as needed.
+        const Entry& e = ents[X * kRing + k];
+        const int kind = e.kind;
+        const int flags = e.flags;
+        if (kind == kEnd) {
+          mbar_arrive(bar_e_empty(X, k));
+          ++rc;
+          run = false;
+          break;
         }
-        mbar_arrive(bar_i_empty(is));
-        if (!warp_wait(bar_s_full(it & 1), (it >> 1) & 1, abort_flag, p.status)) {
-          ok = false;
+        const int ns = e.ns;
+        uint32_t vmask = 0u, dmask = 0u;   // key blocks this row sees; diagonal blocks
+        if (first) {
+          bh = e.bh;
+          qb = e.Qt * 4 + qw;
+          i = qb * 32 + lane;
+          if (!C::kAttn && qb < p.nq)
+            lse_l2 = p.lse_in[(long long)bh * p.n + i] * 1.4426950408889634f;
+        }
+#pragma unroll
+        for (int s = 0; s < kSlots; ++s) {
+          if (s < ns && ((e.own[s] >> qw) & 1)) {
+            vmask |= 1u << s;
+            if (e.kb[s] == qb) dmask |= 1u << s;
+          }
+        }
+        if (!warp_wait(bar_s_full(X), cnt & 1, abort_flag, p.status)) {
+          run = false;
           break;
         }
         tc_fence_after();
-        uint32_t sr[2][32];
-#pragma unroll
-        for (int x = 0; x < 2; ++x)
-          if (vld[x]) tmem_ld32(t_row + (it & 1) * 128 + (2 * half + x) * 32, sr[x]);
-        tmem_wait_ld();
-        reg_fence(sr[0]);
-        reg_fence(sr[1]);
+        ++cnt;
+
         if (!C::kAttn) {
-          tc_fence_before();
-          mbar_arrive(bar_s_free(it & 1));
-          // ---------------- block mass: sum_j exp(s_ij*scale - lse_i) over the block, mean over rows
-          float acc[2];
-#pragma unroll
-          for (int x = 0; x < 2; ++x) {
+          // -------- block mass: sum_j 2^(s_ij*scale*log2e - lse_i*log2e), mean over rows
+#pragma unroll 1
+          for (int s = 0; s < kSlots; ++s) {
+            if (!((vmask >> s) & 1u)) continue;
+            uint32_t v[32];
+            tmem_ld32(t_lane + s_col + s * 32, v);
+            tmem_wait_ld();
+            reg_fence(v);
             float a4[4] = {0.f, 0.f, 0.f, 0.f};
-            if (vld[x]) {
-              if (kbs[x] == qb) {
+            const bool diag = (dmask >> s) & 1u;
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                  const float e = fast_exp2(fmaf(__uint_as_float(sr[x][c]), sl2, -lse_l2));
-                  a4[c & 3] += (c > lane) ? 0.f : e;
-                }
-              } else {
+            for (int c = 0; c < 32; ++c) {
+              const float ev = fast_exp2(fmaf(__uint_as_float(v[c]), sl2, -lse_l2));
+              a4[c & 3] += (diag && c > lane) ? 0.f : ev;
+            }
+            // the warp's 32 lanes are the 32 rows of query block qb
+            float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (lane == 0) p.mass[((long long)bh * p.nq + qb) * p.nq + e.kb[s]] = acc * (1.0f / 32.0f);
+          }
+          tc_fence_before();
+          mbar_arrive(bar_s_free(X));
+          mbar_arrive(bar_e_empty(X, k));
+          ++rc;
+          first = false;
+          if (flags & kLast) break;
+          continue;
+        }
+
+        // -------- pass 1: row max over the visible key blocks (log2 domain), two blocks
+        // per TMEM round trip
+        float mx;
+        {
+          float mxa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+          for (int s0 = 0; s0 < kSlots; s0 += 2) {
+            uint32_t sr[2][32];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              if ((vmask >> (s0 + h)) & 1u) tmem_ld32(t_lane + s_col + (s0 + h) * 32, sr[h]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (!((vmask >> (s0 + h)) & 1u)) continue;
+              reg_fence(sr[h]);
+              if ((dmask >> (s0 + h)) & 1u) {
 #pragma unroll
                 for (int c = 0; c < 32; ++c)
-                  a4[c & 3] += fast_exp2(fmaf(__uint_as_float(sr[x][c]), sl2, -lse_l2));
+                  if (c > lane) sr[h][c] = __float_as_uint(-INFINITY);
               }
-            }
-            acc[x] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-          }
-          // the warp's 32 lanes are the 32 rows of query block qb: two interleaved butterflies
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], o);
-            acc[1] += __shfl_xor_sync(0xffffffffu, acc[1], o);
-          }
-          if (lane < 2) {
-            const float mine = lane == 0 ? acc[0] : acc[1];
-            const int kbl = lane == 0 ? kbs[0] : kbs[1];
-            const int v = lane == 0 ? vld[0] : vld[1];
-            if (v) p.mass[((long long)bh * p.nq + qb) * p.nq + kbl] = mine * (1.0f / 32.0f);
-          }
-        } else {
-          // ---------------- online softmax of this half (log2 domain, lazily rescaled)
-          // Slot validity and the diagonal are warp-uniform branches.  Packed f32x2
-          // FMA/ADD and 3-input max keep the instruction count per element low.
-#pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            if (vld[x] && kbs[x] == qb) {
-#pragma unroll
-              for (int c = 0; c < 32; ++c)
-                if (c > lane) sr[x][c] = __float_as_uint(-INFINITY);
-            }
-          }
-          float mxa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            if (vld[x]) {
 #pragma unroll
               for (int c = 0; c < 32; c += 8) {
 #pragma unroll
                 for (int y = 0; y < 4; ++y)
-                  mxa[y] = max3(mxa[y], __uint_as_float(sr[x][c + 2 * y]),
-                                __uint_as_float(sr[x][c + 2 * y + 1]));
+                  mxa[y] = max3(mxa[y], __uint_as_float(sr[h][c + 2 * y]),
+                                __uint_as_float(sr[h][c + 2 * y + 1]));
               }
             }
           }
-          const float mx = max3(mxa[0], mxa[1], fmaxf(mxa[2], mxa[3])) * sl2;
-          const float m_new = fmaxf(m, mx);
-          const bool need = m_new > m + 8.0f;   // true on the first finite score
-          const bool warp_need = __any_sync(0xffffffffu, need);
-          const float m_use = warp_need ? m_new : m;
-          const float alpha = (warp_need && m != -INFINITY) ? fast_exp2(m - m_use) : 1.0f;
-          const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;  // all scores are -inf then
-          const uint64_t sc2 = f2(sl2, sl2), nm2 = f2(neg_m, neg_m);
-          float ps[2] = {0.f, 0.f};   // per-slot sums of this row's probabilities
-          // P of slot x, keys 2c' and 2c'+1 as one bf16 pair, goes to sr[x][c'] (already consumed)
-#pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            if (vld[x]) {
-              uint64_t rs2[2] = {0ull, 0ull};
-#pragma unroll
-              for (int c = 0; c < 32; c += 2) {
-                float t0, t1;
-                f2_split(fma2(f2(__uint_as_float(sr[x][c]), __uint_as_float(sr[x][c + 1])), sc2, nm2),
-                         t0, t1);
-                const float e0 = fast_exp2(t0), e1 = fast_exp2(t1);
-                rs2[(c >> 1) & 1] = add2(rs2[(c >> 1) & 1], f2(e0, e1));
-                sr[x][c >> 1] = pack_bf16x2(e0, e1);
-              }
-              float lo, hi;
-              f2_split(add2(rs2[0], rs2[1]), lo, hi);
-              ps[x] = lo + hi;
-            } else {
-#pragma unroll
-              for (int c = 0; c < 16; ++c) sr[x][c] = 0u;   // not this warp's block: P = 0
-            }
-          }
-          const float rs = ps[0] + ps[1];
-          if (MODE == kModeDense && p.blse != nullptr) {
-            // block log-sum-exp of this row over each owned key block, log2 domain:
-            // blse = m + log2(sum_j 2^(s_ij*scale*log2e - m)); the mass pass turns it into
-            // block mass with the final lse.  Layout [bh][key block][row]: 32 lanes store
-            // 32 consecutive floats.
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-              if (vld[x])
-                p.blse[((long long)bh * p.nq + kbs[x]) * p.n + i] =
-                    ps[x] > 0.f ? m_use + __log2f(ps[x]) : -INFINITY;
-            }
-          }
-          l = l * alpha + rs;
-          m = m_use;
-          if (warp_need && started) {
-            // O of this half is rescaled in place: its previous PV must have finished.
-            if (!warp_wait(bar_o_done((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, p.status)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < D / 16; ++c) {
-              uint32_t o[16];
-              tmem_ld16(t_row + o_col + c * 16, o);
-              tmem_wait_ld();
-              reg_fence(o);
-#pragma unroll
-              for (int y = 0; y < 16; ++y) o[y] = __float_as_uint(__uint_as_float(o[y]) * alpha);
-              tmem_st16(t_row + o_col + c * 16, o);
-            }
-          }
-          // P -> TMEM over the first 32 columns of this half's part of S buffer it&1
-          tmem_st32_halves(t_row + (it & 1) * 128 + 64 * half, sr[0], sr[1]);
-          tmem_wait_st();
-          if (2 * ns > 4 * half) started = true;
-          if (2 * ns > 4 * (1 - half)) wrote_other = true;
-          tc_fence_before();
-          mbar_arrive(bar_p_full(half, it & 1));
+          mx = max3(mxa[0], mxa[1], fmaxf(mxa[2], mxa[3])) * sl2;
         }
-        ++it;
-        if (last) break;
-      }
-      if (!ok) break;
+        const float m_new = fmaxf(m, mx);
+        const bool need = m_new > m + 8.0f;   // true on the first finite score
+        const bool warp_need = __any_sync(0xffffffffu, need);
+        const float m_use = warp_need ? m_new : m;
+        const float alpha = (warp_need && m != -INFINITY) ? fast_exp2(m - m_use) : 1.0f;
+        const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;  // all scores are -inf then
+        const uint64_t sc2 = f2(sl2, sl2), nm2 = f2(neg_m, neg_m);
 
-      if (C::kAttn) {
-        // ---------------- epilogue: merge the halves, O -> bf16 -> smem (Q tile) -> TMA store
-        if (!warp_wait(bar_o_done((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // exchange (m, l) with the other half's thread of the same row (P buffer is idle now)
-        xchg[(half * 128 + r) * 2 + 0] = m;
-        xchg[(half * 128 + r) * 2 + 1] = l;
-        mbar_arrive(bar_merge);
-        if (!warp_wait(bar_merge, tl & 1, abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
-        const float m_o = xchg[((1 - half) * 128 + r) * 2 + 0];
-        const float l_o = xchg[((1 - half) * 128 + r) * 2 + 1];
-        const float ma = half == 0 ? m : m_o, la = half == 0 ? l : l_o;
-        const float mb = half == 0 ? m_o : m, lb = half == 0 ? l_o : l;
-        const bool a_written = half == 0 ? started : wrote_other;
-        const bool b_written = half == 0 ? wrote_other : started;
-        const float mt = fmaxf(ma, mb);
-        const float sa = (la > 0.f) ? fast_exp2(ma - mt) : 0.f;
-        const float sb = (lb > 0.f) ? fast_exp2(mb - mt) : 0.f;
-        const float L = la * sa + lb * sb;
-        const float inv = L > 0.f ? 1.0f / L : 0.f;
-        const float ca = sa * inv, cb = sb * inv;
-        // this half writes output columns [half*D/2, (half+1)*D/2)
+        // -------- pass 2: P = 2^(s*scale*log2e - m) as bf16 pairs over S_X columns [0, 64)
+        // Key block s goes to P columns [16 s, 16 s + 16), which lie in S columns of
+        // blocks <= s that this pass has already read.
+        float rs = 0.f;
+        auto block_exp = [&](uint32_t (&v)[32], int s) {
+          uint32_t w[16];
+          if ((vmask >> s) & 1u) {
+            reg_fence(v);
+            if ((dmask >> s) & 1u) {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          const int col0 = half * (D / 2) + c * 16;
-          uint32_t oa[16], ob[16];
-#pragma unroll
-          for (int y = 0; y < 16; ++y) oa[y] = ob[y] = 0u;
-          if (a_written) tmem_ld16(t_row + C::kOCol + col0, oa);
-          if (b_written) tmem_ld16(t_row + C::kOCol + 128 + col0, ob);
-          tmem_wait_ld();
-          reg_fence(oa);
-          reg_fence(ob);
-#pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {
-            const int cabs = col0 + ch * 8;
-            const int pnl = cabs >> 6;
-            const int cc = (cabs & 63) >> 3;
-            uint32_t w[4];
-#pragma unroll
-            for (int y = 0; y < 4; ++y) {
-              const int e0 = ch * 8 + 2 * y;
-              const float v0 = __uint_as_float(oa[e0]) * ca + __uint_as_float(ob[e0]) * cb;
-              const float v1 = __uint_as_float(oa[e0 + 1]) * ca + __uint_as_float(ob[e0 + 1]) * cb;
-              w[y] = pack_bf16x2(v0, v1);
+              for (int c = 0; c < 32; ++c)
+                if (c > lane) v[c] = __float_as_uint(-INFINITY);
             }
-            const uint32_t addr = sQ + pnl * kPanelBytes + r * kPanelRowBytes + ((cc ^ (r & 7)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]),
-                         "r"(w[2]), "r"(w[3])
-                         : "memory");
-          }
-        }
-        if (half == 0 && p.lse != nullptr && i < p.n)
-          p.lse[(long long)bh * p.n + i] =
-              L > 0.f ? (mt + __log2f(L)) * 0.6931471805599453f : -INFINITY;
-        tc_fence_before();
-        fence_proxy_async_smem();
-        mbar_arrive(bar_o_staged);
-        if (warp == 3 && lane == 0) {
-          if (!mbar_wait(bar_o_staged, tl & 1, abort_flag, p.status)) {
-            ok = false;
+            uint64_t rs2[2] = {0ull, 0ull};
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              float t0, t1;
+              f2_split(fma2(f2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), sc2, nm2), t0, t1);
+              const float e0 = fast_exp2(t0), e1 = fast_exp2(t1);
+              rs2[(c >> 1) & 1] = add2(rs2[(c >> 1) & 1], f2(e0, e1));
+              w[c >> 1] = pack_bf16x2(e0, e1);
+            }
+            float lo, hi;
+            f2_split(add2(rs2[0], rs2[1]), lo, hi);
+            const float ps = lo + hi;
+            rs += ps;
+            if (MODE == kModeDense && p.blse != nullptr) {
+              // block log-sum-exp of this row over key block kb, log2 domain:
+              // blse = m + log2(sum_j 2^(s_ij*scale*log2e - m)); the mass pass turns it
+              // into block mass with the final lse.  Layout [bh][key block][row]: 32
+              // lanes store 32 consecutive floats.
+              p.blse[((long long)bh * p.nq + e.kb[s]) * p.n + i] =
+                  ps > 0.f ? m_use + __log2f(ps) : -INFINITY;
+            }
           } else {
-            for (int pn = 0; pn < C::kPanels; ++pn)
-              tma_store_3d(&tmO, sQ + pn * kPanelBytes, pn * 64, Qt * kBM, bh);
-            bulk_commit_group();
-            bulk_wait_group_read0();
-            mbar_arrive(bar_q_empty);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) w[c] = 0u;   // not this row's block (or unused): P = 0
+          }
+          tmem_st16(t_lane + s_col + s * 16, w);
+        };
+#pragma unroll 1
+        for (int s = 0; s < kSlots; ++s) {
+          uint32_t v[32];
+          if ((vmask >> s) & 1u) {
+            tmem_ld32(t_lane + s_col + s * 32, v);
+            tmem_wait_ld();
+          }
+          block_exp(v, s);
+        }
+        if (warp_need && !first) {
+          // O_X is rescaled in place.  Its last PV has completed: QK_X of this entry
+          // was issued only after it.
+#pragma unroll 1
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(t_lane + o_col + c * 16, o);
+            tmem_wait_ld();
+            reg_fence(o);
+#pragma unroll
+            for (int y = 0; y < 16; ++y) o[y] = __float_as_uint(__uint_as_float(o[y]) * alpha);
+            tmem_st16(t_lane + o_col + c * 16, o);
           }
         }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (!ok) *abort_flag = 1;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_p_full(X));
+        mbar_arrive(bar_e_empty(X, k));
+        ++rc;
+        l = l * alpha + rs;
+        m = m_use;
+        first = false;
+        if (flags & kLast) break;
       }
+      if (!run || !C::kAttn) continue;
+
+      // ---------------- epilogue: O_X / l -> bf16 -> global rows (one row per thread)
+      if (!warp_wait(bar_o_done(X), (cnt - 1) & 1, abort_flag, p.status)) break;
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.0f / l : 0.f;
+      if (qb < p.nq) {
+        uint8_t* orow = static_cast<uint8_t*>(p.o) + ((long long)bh * p.n + i) * (D * 2);
+#pragma unroll 1
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t o[16];
+          tmem_ld16(t_lane + o_col + c * 16, o);
+          tmem_wait_ld();
+          reg_fence(o);
+          uint32_t w[8];
+#pragma unroll
+          for (int y = 0; y < 8; ++y)
+            w[y] = pack_bf16x2(__uint_as_float(o[2 * y]) * inv, __uint_as_float(o[2 * y + 1]) * inv);
+          st_global_v4(orow + c * 32, w[0], w[1], w[2], w[3]);
+          st_global_v4(orow + c * 32 + 16, w[4], w[5], w[6], w[7]);
+        }
+        if (p.lse != nullptr)
+          p.lse[(long long)bh * p.n + i] =
+              l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+      }
+      tc_fence_before();
+      mbar_arrive(bar_o_free(X));
     }
-    if (C::kAttn && warp == 3 && lane == 0) bulk_wait_group0();
   }
 
   tc_fence_before();
@@ -803,39 +881,47 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, int MODE>
 static cudaError_t launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                               const CUtensorMap& to, const AttnParams& p, int grid,
-                               cudaStream_t stream) {
+                               const AttnParams& p, int grid, cudaStream_t stream,
+                               const char** why) {
   using C = Cfg<D, MODE>;
   static bool configured = false;  // per instantiation; attribute is per function
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, MODE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    // The setmaxnreg split assumes the launch allocates kLaunchRegs per thread.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_kernel<D, MODE>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kLaunchRegs) {
+      *why = "attention kernel register count differs from its setmaxnreg split";
+      return cudaErrorInvalidKernelImage;
+    }
+    e = cudaFuncSetAttribute(attn_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  attn_kernel<D, MODE><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+  attn_kernel<D, MODE><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
 template <int MODE>
 static cudaError_t launch_mode(int d, const CUtensorMap& tq, const CUtensorMap& tk,
-                               const CUtensorMap& tv, const CUtensorMap& to, const AttnParams& p,
-                               int grid, cudaStream_t stream) {
+                               const CUtensorMap& tv, const AttnParams& p, int grid,
+                               cudaStream_t stream, const char** why) {
   switch (d) {
-    case 64: return launch_impl<64, MODE>(tq, tk, tv, to, p, grid, stream);
-    case 96: return launch_impl<96, MODE>(tq, tk, tv, to, p, grid, stream);
-    case 128: return launch_impl<128, MODE>(tq, tk, tv, to, p, grid, stream);
+    case 64: return launch_impl<64, MODE>(tq, tk, tv, p, grid, stream, why);
+    case 96: return launch_impl<96, MODE>(tq, tk, tv, p, grid, stream, why);
+    case 128: return launch_impl<128, MODE>(tq, tk, tv, p, grid, stream, why);
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_attention(int mode, int d, const CUtensorMap& tq, const CUtensorMap& tk,
-                             const CUtensorMap& tv, const CUtensorMap& to, const AttnParams& p,
-                             int grid, cudaStream_t stream) {
+                             const CUtensorMap& tv, const AttnParams& p, int grid,
+                             cudaStream_t stream, const char** why) {
   switch (mode) {
-    case kModeDense: return launch_mode<kModeDense>(d, tq, tk, tv, to, p, grid, stream);
-    case kModeSparse: return launch_mode<kModeSparse>(d, tq, tk, tv, to, p, grid, stream);
-    case kModeMass: return launch_mode<kModeMass>(d, tq, tk, tv, to, p, grid, stream);
+    case kModeDense: return launch_mode<kModeDense>(d, tq, tk, tv, p, grid, stream, why);
+    case kModeSparse: return launch_mode<kModeSparse>(d, tq, tk, tv, p, grid, stream, why);
+    case kModeMass: return launch_mode<kModeMass>(d, tq, tk, tv, p, grid, stream, why);
   }
   return cudaErrorInvalidValue;
 }

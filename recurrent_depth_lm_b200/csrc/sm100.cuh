@@ -57,25 +57,66 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that lets the thread sleep until the phase completes or suspend_ns
+// nanoseconds pass (the suspend-time hint of mbarrier.try_wait), so that waiting
+// warps do not take issue slots from the warps that compute.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Suspend-time hint of a pipeline wait: long enough that a waiting warp sleeps
+// through a whole pipeline stage, short enough to notice an abort promptly.
+constexpr uint32_t kSuspendNs = 20000u;
+
 // Wait for the phase with the given parity to complete.  Gives up after
-// limit_ns (default kWaitLimitNs), or at once if *abort is set by another role; on giving up it
-// ORs kStatusTimeout into *status, sets *abort and returns false.
+// limit_ns (default kWaitLimitNs) of %globaltimer, or as soon as *abort (a flag in
+// shared memory) is set by another role; on giving up it ORs kStatusTimeout into
+// *status, sets *abort and returns false.  One compact PTX block per wait site: the
+// polling try_wait carries the suspend-time hint so a waiting warp sleeps.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           unsigned int* status,
                                           unsigned long long limit_ns = kWaitLimitNs) {
-  if (mbar_try_wait(bar, parity)) return true;
-  unsigned long long t0 = globaltimer();
-  for (uint32_t spin = 1;; ++spin) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((spin & 255u) == 0) {
-      if (*abort) return false;
-      if (globaltimer() - t0 > limit_ns) {
-        atomicOr(status, kStatusTimeout);
-        *abort = 1;
-        return false;
-      }
-    }
-  }
+  uint32_t ok;
+  asm volatile(
+      "{\n\t"
+      ".reg .pred p, q;\n\t"
+      ".reg .u64 t0, t1;\n\t"
+      ".reg .u32 a;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "@p bra WAIT_OK;\n\t"
+      "mov.u64 t0, %%globaltimer;\n\t"
+      "WAIT_LOOP:\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "@p bra WAIT_OK;\n\t"
+      "ld.volatile.shared.u32 a, [%4];\n\t"
+      "setp.ne.u32 q, a, 0;\n\t"
+      "@q bra WAIT_FAIL;\n\t"
+      "mov.u64 t1, %%globaltimer;\n\t"
+      "sub.u64 t1, t1, t0;\n\t"
+      "setp.le.u64 q, t1, %5;\n\t"
+      "@q bra WAIT_LOOP;\n\t"
+      "red.or.b32 [%6], %7;\n\t"
+      "st.volatile.shared.u32 [%4], 1;\n\t"
+      "WAIT_FAIL:\n\t"
+      "mov.u32 %0, 0;\n\t"
+      "bra WAIT_END;\n\t"
+      "WAIT_OK:\n\t"
+      "mov.u32 %0, 1;\n\t"
+      "WAIT_END:\n\t"
+      "}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(kSuspendNs), "r"(smem_u32((const void*)abort)), "l"(limit_ns),
+        "l"(status), "r"(kStatusTimeout)
+      : "memory");
+  return ok != 0;
 }
 
 // ---------------------------------------------------------------- proxies / fences
@@ -167,6 +208,43 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Warp-collective forms: the whole (converged) warp executes the instruction and
+// one lane chosen by elect.sync issues it.  Keeping the issuing warp converged lets
+// the descriptor arithmetic stay warp-uniform.
+__device__ __forceinline__ void mma_bf16_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_bf16_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit_warp(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          bar)
+      : "memory");
+}
+
+// One arrival on `bar` from a converged warp (one elected lane arrives).
+__device__ __forceinline__ void mbar_arrive_warp(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b64 st;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e mbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar)
       : "memory");
 }
 

@@ -17,6 +17,7 @@ struct AttnParams {
   int nq;               // n / 32
   int num_tiles;        // BH * ceil(nq / 4)
   float scale_log2;     // softmax scale * log2(e)
+  void* o;              // [BH, n, d] bf16 output (dense / sparse)
   float* lse;           // [BH, n] output (dense / sparse), nullable
   const float* lse_in;  // [BH, n] input (mass mode)
   float* mass;          // [BH, nq, nq] output (mass mode)
@@ -27,9 +28,10 @@ struct AttnParams {
   unsigned int* status;        // device status word
 };
 
+// On a launch-configuration failure specific to the kernel, *why gets a description.
 cudaError_t launch_attention(int mode, int d, const CUtensorMap& tq, const CUtensorMap& tk,
-                             const CUtensorMap& tv, const CUtensorMap& to, const AttnParams& p,
-                             int grid, cudaStream_t stream);
+                             const CUtensorMap& tv, const AttnParams& p, int grid,
+                             cudaStream_t stream, const char** why);
 int attention_smem_bytes(int mode, int d);
 
 // mass[bh][q][b] = (1/32) sum_{i in q} 2^(blse[bh][b][i] - lse[bh][i] * log2 e), b <= q
