@@ -186,8 +186,9 @@ int wise_build_schedule_static(const uint32_t* union_bits, int32_t* row_offsets,
  * row_offsets, col_idx : the schedule (see wise_build_schedule); each row's
  *               indices must be ascending and <= its query block.  Entries
  *               outside [0, col_count) or violating that order are skipped and
- *               flag WISE_STATUS_BAD_SCHEDULE; they never cause an out-of-range
- *               access.
+ *               flag WISE_STATUS_BAD_SCHEDULE; a row whose offsets are not
+ *               ascending within [0, col_count] is treated as empty and flagged.
+ *               Neither causes an out-of-range access.
  * col_count   : number of valid entries in col_idx (row_offsets[B*H*nq]).
  * lse         : fp32 [B, H, n] output or NULL.
  * A row whose schedule row is empty gets O = 0 and lse = -inf.

@@ -54,15 +54,6 @@ constexpr int kPanelBytes = kBM * kPanelRowBytes;  // one 128-row panel = 16 KB
 constexpr int kMaxWords = 16;   // schedule bitmask words per query block (nq <= 512)
 constexpr int kRing = 4;        // work entries in flight per tile slot
 
-// Register split (setmaxnreg): the launch gives every thread kLaunchRegs; the
-// control warpgroup (TMA producers, MMA issuer) drops to kCtlRegs and the two
-// softmax warpgroups rise to kSoftRegs.  The sum must not exceed the launch's.
-constexpr int kLaunchRegs = 168;
-constexpr int kCtlRegs = 72;
-constexpr int kSoftRegs = 216;
-static_assert(128 * kCtlRegs + 256 * kSoftRegs <= kLaunchRegs * kThreads, "register split");
-static_assert(kLaunchRegs * kThreads <= 65536, "register file");
-
 enum : int { kWork = 0, kEnd = 1 };
 enum : int { kFirst = 1, kLast = 2 };
 
@@ -167,32 +158,54 @@ struct MaskList {
   }
 };
 
-// Build the 4 per-row bitmasks of a sparse tile (whole producer warp).  Entries
-// outside [0, q] or outside col_idx[0, col_count) are dropped and flagged.
+// Build the 4 per-row bitmasks of a sparse tile (whole producer warp).  The tile's
+// rows are consecutive in the CSR arrays: when their offsets are ascending within
+// [0, col_count], one strided pass over col_idx[row_offsets[r0], row_offsets[r0 + nr])
+// covers them.  Otherwise each row is taken on its own and a row with bad offsets
+// is dropped.  Entries outside [0, q] are dropped.  Anything dropped is flagged.
 __device__ void build_tile_masks(uint32_t* mask, const AttnParams& p, int bh, int Qt, int lane) {
   const int words = (p.nq + 31) / 32;
   for (int x = lane; x < 4 * kMaxWords; x += 32) mask[x] = 0u;
+  const int qb0 = Qt * 4;
+  const int nr = min(4, p.nq - qb0);                 // rows of this tile
+  const long long row0 = (long long)bh * p.nq + qb0;
+  // offsets of rows r0 .. r0 + nr in lanes 0 .. nr (one load each)
+  const long long off = lane <= nr ? (long long)p.row_offsets[row0 + lane] : 0;
+  const long long o1 = __shfl_sync(0xffffffffu, off, min(1, nr));
+  const long long o2 = __shfl_sync(0xffffffffu, off, min(2, nr));
+  const long long o3 = __shfl_sync(0xffffffffu, off, min(3, nr));
+  const long long nxt = __shfl_down_sync(0xffffffffu, off, 1);
+  // lane r < nr checks row r: 0 <= beg <= end <= col_count
+  const bool row_bad = lane < nr && (off < 0 || nxt < off || nxt > p.col_count);
+  bool bad = false;
   __syncwarp();
-  for (int r = 0; r < 4; ++r) {
-    const int qb = Qt * 4 + r;
-    if (qb >= p.nq) break;
-    const long long row = (long long)bh * p.nq + qb;
-    long long beg = p.row_offsets[row];
-    long long end = p.row_offsets[row + 1];
-    bool bad = false;
-    if (beg < 0 || end > p.col_count || beg > end) {
-      bad = true;
-      beg = end = 0;
-    }
+  if (!__any_sync(0xffffffffu, row_bad)) {
+    const long long beg = __shfl_sync(0xffffffffu, off, 0);
+    const long long end = __shfl_sync(0xffffffffu, off, nr);
     for (long long e = beg + lane; e < end; e += 32) {
+      const int r = (e >= o1) + (e >= o2) + (e >= o3);   // row of entry e
+      const int qb = qb0 + r;
       const int kb = p.col_idx[e];
       if (kb >= 0 && kb <= qb && kb < words * 32)
         atomicOr(&mask[r * kMaxWords + (kb >> 5)], 1u << (kb & 31));
       else
         bad = true;
     }
-    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.status, kStatusBadSchedule);
+  } else {
+    bad = true;
+    for (int r = 0; r < nr; ++r) {
+      const long long beg = __shfl_sync(0xffffffffu, off, r);
+      const long long end = __shfl_sync(0xffffffffu, nxt, r);
+      if (__shfl_sync(0xffffffffu, row_bad ? 1 : 0, r)) continue;
+      const int qb = qb0 + r;
+      for (long long e = beg + lane; e < end; e += 32) {
+        const int kb = p.col_idx[e];
+        if (kb >= 0 && kb <= qb && kb < words * 32)
+          atomicOr(&mask[r * kMaxWords + (kb >> 5)], 1u << (kb & 31));
+      }
+    }
   }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.status, kStatusBadSchedule);
   __syncwarp();
 }
 
@@ -331,10 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  // Each setmaxnreg sits at the head of its warpgroup's branch, so that the code of
-  // every role is dominated by the register limit that applies to it.
   if (warp < 4) {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtlRegs));
   if (warp == 0) {
     // ======================================================= Q / K producer, entry writer
     if (lane == 0) {
@@ -552,10 +562,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t p_tmem = tmem_base + X * 128;
         const uint32_t o_tmem = tmem_base + C::kOCol + X * 128;
         const int nk = 2 * S.pend_ns;
-        for (int kk = 0; kk < nk; ++kk) {
-          const uint64_t b = smem_desc_sw128(vbase + kk * 16 * kPanelRowBytes, kPanelBytes, 1024);
-          mma_bf16_ts_warp(o_tmem, p_tmem + kk * 8, b, idesc_o, (S.pend_first && kk == 0) ? 0u : 1u);
-        }
+        // descriptor start addresses advance by 16 keys = 2048 bytes (>> 4 = 128) per step
+        const uint64_t b0 = smem_desc_sw128(vbase, kPanelBytes, 1024);
+        for (int kk = 0; kk < nk; ++kk)
+          mma_bf16_ts_warp(o_tmem, p_tmem + kk * 8, b0 + (uint64_t)(kk * 128), idesc_o,
+                           (S.pend_first && kk == 0) ? 0u : 1u);
         mma_commit_warp(bar_o_done(X));
         mma_commit_warp(bar_v_empty(vs));
         ++S.pvc;
@@ -601,11 +612,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_tmem = tmem_base + X * 128;
         const uint32_t qbase = sQ + X * C::kTileBytes;
         const uint32_t kbase = sK + ks * C::kTileBytes;
+        // K steps of 16 columns: +32 bytes within a 64-column panel, then the next panel;
+        // the descriptors' start fields (address >> 4) advance by the same offsets >> 4
+        const uint64_t a0 = smem_desc_sw128(qbase, 16, 1024);
+        const uint64_t b0 = smem_desc_sw128(kbase, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
-          mma_bf16_ss_warp(d_tmem, smem_desc_sw128(qbase + off, 16, 1024),
-                           smem_desc_sw128(kbase + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((kk >> 2) * kPanelBytes + (kk & 3) * 32) >> 4);
+          mma_bf16_ss_warp(d_tmem, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
         }
         mma_commit_warp(bar_s_full(X));
         mma_commit_warp(bar_k_empty(ks));
@@ -636,7 +650,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftRegs));
     // ======================================================= softmax / epilogue of slot X
     // Thread = row.  Each iteration reads its key blocks from S_X twice (row max,
     // then exponentials), one 32-column block at a time in a rolled loop: the hot
@@ -886,16 +899,8 @@ static cudaError_t launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, con
   using C = Cfg<D, MODE>;
   static bool configured = false;  // per instantiation; attribute is per function
   if (!configured) {
-    // The setmaxnreg split assumes the launch allocates kLaunchRegs per thread.
-    cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, attn_kernel<D, MODE>);
-    if (e != cudaSuccess) return e;
-    if (fa.numRegs != kLaunchRegs) {
-      *why = "attention kernel register count differs from its setmaxnreg split";
-      return cudaErrorInvalidKernelImage;
-    }
-    e = cudaFuncSetAttribute(attn_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     configured = true;
   }

@@ -180,6 +180,38 @@ def test_sparse_bad_schedule_entries_are_skipped(ops):
     compare_o(o, o_ref)
 
 
+def test_sparse_bad_row_offsets_are_empty_rows(ops):
+    """A row whose offsets are not ascending within [0, col_count] is empty and flagged;
+    its neighbour, whose range then covers foreign entries, keeps only entries <= q."""
+    b, h, n, d = 1, 1, 256, 64
+    nq = n // 32
+    qb, kb, vb = rand_qkv_bits(b, h, n, d, seed=17)
+    sup = np.tril(np.ones((nq, nq), dtype=bool))
+    ro, ci, nnz = csr_device([sup])
+    ro_h = ro.cpu().numpy().copy()
+    ci_h = ci.cpu().numpy()
+    ro_h[4] = ro_h[5] + 3          # row 4 ends before it begins; row 3 now spans into row 4's entries
+    expect = np.zeros_like(sup)
+    for r in range(nq):
+        beg, end = int(ro_h[r]), int(ro_h[r + 1])
+        if beg < 0 or end < beg or end > nnz:
+            continue
+        for e in range(beg, end):
+            if 0 <= ci_h[e] <= r:
+                expect[r, ci_h[e]] = True
+    assert not expect[4].any() and expect[3].sum() == 4
+    ops.device_status(clear=True)
+    o, _ = ops.sparse_attn(to_dev(qb), to_dev(kb), to_dev(vb),
+                           torch.tensor(ro_h, dtype=torch.int32, device="cuda"), ci, nnz)
+    st = ops.device_status(clear=True)
+    assert st & 0x2
+    o = dev_f32(o)[0, 0]
+    o_ref, _ = O.masked_attention(*(bf16_bits_to_f64(x[0, 0]) for x in (qb, kb, vb)), expect)
+    rows = np.repeat(expect.any(axis=1), 32)       # the empty row 4 has no softmax: O = 0
+    compare_o(o[rows], o_ref[rows])
+    assert np.all(o[~rows] == 0.0)
+
+
 @pytest.mark.parametrize("nq,bh", [(8, 2), (37, 3), (128, 2), (512, 1)])
 def test_select_union_matches_oracle(ops, nq, bh):
     rng = np.random.default_rng(nq)
