@@ -182,14 +182,25 @@ __device__ void build_tile_masks(uint32_t* mask, const AttnParams& p, int bh, in
   if (!__any_sync(0xffffffffu, row_bad)) {
     const long long beg = __shfl_sync(0xffffffffu, off, 0);
     const long long end = __shfl_sync(0xffffffffu, off, nr);
-    for (long long e = beg + lane; e < end; e += 32) {
-      const int r = (e >= o1) + (e >= o2) + (e >= o3);   // row of entry e
-      const int qb = qb0 + r;
-      const int kb = p.col_idx[e];
-      if (kb >= 0 && kb <= qb && kb < words * 32)
-        atomicOr(&mask[r * kMaxWords + (kb >> 5)], 1u << (kb & 31));
-      else
-        bad = true;
+    // 8 entries per lane per round: all loads are issued before any is used
+    for (long long e0 = beg + lane; e0 < end; e0 += 8 * 32) {
+      int kbs[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const long long e = e0 + u * 32;
+        kbs[u] = e < end ? p.col_idx[e] : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const long long e = e0 + u * 32;
+        if (e >= end) break;
+        const int r = (e >= o1) + (e >= o2) + (e >= o3);   // row of entry e
+        const int kb = kbs[u];
+        if (kb >= 0 && kb <= qb0 + r && kb < words * 32)
+          atomicOr(&mask[r * kMaxWords + (kb >> 5)], 1u << (kb & 31));
+        else
+          bad = true;
+      }
     }
   } else {
     bad = true;
