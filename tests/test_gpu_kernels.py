@@ -76,6 +76,28 @@ def test_dense_without_lse(ops):
         compare_o(o[0, hi], o_ref)
 
 
+# More tiles than 2 x 148 tile slots: every CTA cycles both of its tile slots through
+# several query tiles (tile switches, slot end markers, uneven slot progress).
+MANY_TILES = [(2, 160, 256, 64), (1, 80, 512, 128), (1, 100, 384, 96)]
+
+
+@pytest.mark.parametrize("b,h,n,d", MANY_TILES)
+def test_dense_many_tiles_per_cta(ops, b, h, n, d):
+    qb, kb, vb = rand_qkv_bits(b, h, n, d, seed=3 * n + d)
+    o, lse, mass = ops.full_attn_mass(to_dev(qb), to_dev(kb), to_dev(vb), with_mass=True)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    o, lse, mass = dev_f32(o), lse.cpu().numpy(), mass.cpu().numpy()
+    for bi in range(b):
+        for hi in range(h):
+            qf, kf, vf = (bf16_bits_to_f64(x[bi, hi]) for x in (qb, kb, vb))
+            o_ref, lse_ref = O.causal_attention(qf, kf, vf)
+            compare_o(o[bi, hi], o_ref, f"O[{bi},{hi}]")
+            assert np.abs(lse[bi, hi] - lse_ref).max() <= LSE_TOL
+            if hi % 16 == 0:
+                assert np.abs(np.tril(mass[bi, hi]) - O.block_mass(qf, kf)).max() <= MASS_TOL
+
+
 def random_support(nq, rng, p=0.4, diag=True, empty_rows=()):
     s = np.tril(rng.random((nq, nq)) < p)
     if diag:
@@ -116,6 +138,28 @@ def test_sparse_attention_random_schedule(ops, b, h, n, d):
             o_ref, lse_ref = O.masked_attention(qf, kf, vf, sups[bi * h + hi])
             compare_o(o[bi, hi], o_ref, f"sparse O[{bi},{hi}]")
             assert np.abs(lse[bi, hi] - lse_ref).max() <= LSE_TOL
+
+
+@pytest.mark.parametrize("b,h,n,d", MANY_TILES)
+def test_sparse_many_tiles_per_cta(ops, b, h, n, d):
+    nq = n // 32
+    rng = np.random.default_rng(7 + n)
+    qb, kb, vb = rand_qkv_bits(b, h, n, d, seed=5 * n + d)
+    sups = [random_support(nq, rng, p=rng.uniform(0.1, 0.9), empty_rows=(1,) if i % 7 == 0 else ())
+            for i in range(b * h)]
+    ro, ci, nnz = csr_device(sups)
+    o, _ = ops.sparse_attn(to_dev(qb), to_dev(kb), to_dev(vb), ro, ci, nnz)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    o = dev_f32(o)
+    for bi in range(b):
+        for hi in range(h):
+            sup = sups[bi * h + hi]
+            qf, kf, vf = (bf16_bits_to_f64(x[bi, hi]) for x in (qb, kb, vb))
+            o_ref, _ = O.masked_attention(qf, kf, vf, sup)
+            rows = np.repeat(sup.any(axis=1), 32)
+            compare_o(o[bi, hi][rows], o_ref[rows], f"sparse O[{bi},{hi}]")
+            assert np.all(o[bi, hi][~rows] == 0.0)
 
 
 def test_sparse_all_blocks_equals_dense(ops):
