@@ -62,6 +62,11 @@ typedef struct wise_shape {
   int32_t seqlen;
   int32_t head_dim;
   float scale; /* softmax temperature; <= 0 selects 1/sqrt(head_dim) (WISE paper section 3) */
+  /* Heads of K and V (grouped-query attention, as in the Recurrent-Llama geometry of the
+   * WISE paper, section 4: 32 query heads over 8 key/value heads).  0 means kv_heads =
+   * heads.  heads must be a multiple of kv_heads; query head h reads K/V head
+   * h / (heads / kv_heads), and K, V are then [batch, kv_heads, seqlen, head_dim]. */
+  int32_t kv_heads;
 } wise_shape_t;
 
 /*

@@ -34,7 +34,7 @@ ERROR_NAMES = {
 class WiseShape(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("heads", ctypes.c_int32),
                 ("seqlen", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("scale", ctypes.c_float)]
+                ("scale", ctypes.c_float), ("kv_heads", ctypes.c_int32)]
 
 
 class WiseError(RuntimeError):

@@ -121,6 +121,9 @@ int check_shape(const wise_shape_t& s) {
     return fail(WISE_ERR_SHAPE, "head_dim %d unsupported (64, 96 or 128)", s.head_dim);
   const long long bh = (long long)s.batch * s.heads;
   if (bh > (1ll << 24)) return fail(WISE_ERR_SHAPE, "batch*heads %lld too large", bh);
+  if (s.kv_heads < 0 || (s.kv_heads > 0 && s.heads % s.kv_heads != 0))
+    return fail(WISE_ERR_SHAPE, "heads (%d) must be a multiple of kv_heads (%d)", s.heads,
+                s.kv_heads);
   if (!(std::isfinite(s.scale))) return fail(WISE_ERR_ARG, "scale must be finite");
   return WISE_OK;
 }
@@ -137,17 +140,20 @@ int launch_attn(int mode, const void* q, const void* k, const void* v, void* o,
   int rc = device_info(&di);
   if (rc) return rc;
   const int BH = s.batch * s.heads;
+  const int kv = s.kv_heads > 0 ? s.kv_heads : s.heads;
+  const int BHkv = s.batch * kv;
   CUtensorMap tq, tk, tv;
   if ((rc = make_tmap(&tq, q, s.head_dim, s.seqlen, BH, 128))) return rc;
-  if ((rc = make_tmap(&tk, k, s.head_dim, s.seqlen, BH, 32))) return rc;
+  if ((rc = make_tmap(&tk, k, s.head_dim, s.seqlen, BHkv, 32))) return rc;
   if (mode != wise::kModeMass) {
-    if ((rc = make_tmap(&tv, v, s.head_dim, s.seqlen, BH, 32))) return rc;
+    if ((rc = make_tmap(&tv, v, s.head_dim, s.seqlen, BHkv, 32))) return rc;
   } else {
     tv = tk;
   }
   wise::AttnParams p = p0;
   p.o = o;
   p.BH = BH;
+  p.group = s.heads / kv;
   p.n = s.seqlen;
   p.nq = s.seqlen / 32;
   p.num_tiles = BH * ((p.nq + 3) / 4);

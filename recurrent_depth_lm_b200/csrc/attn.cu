@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int pn = 0; pn < C::kPanels; ++pn)
             tma_load_3d(kbase + pn * kPanelBytes + s * 32 * kPanelRowBytes, &tmK, bar_k_full(ks),
-                        pn * 64, kb * 32, S.bh);
+                        pn * 64, kb * 32, S.bh / p.group);
         }
       }
       ++S.rc;
@@ -517,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int pn = 0; pn < C::kPanels; ++pn)
             tma_load_3d(vbase + pn * kPanelBytes + s * 32 * kPanelRowBytes, &tmV, bar_v_full(vs),
-                        pn * 64, kb * 32, bh);
+                        pn * 64, kb * 32, bh / p.group);
         }
         issued = g + 1;
         return true;

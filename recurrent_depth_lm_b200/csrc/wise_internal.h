@@ -13,6 +13,7 @@ enum { kModeDense = 0, kModeSparse = 1, kModeMass = 2 };
 
 struct AttnParams {
   int BH;               // batch * heads
+  int group;            // query heads per K/V head: K/V head of bh is bh / group
   int n;                // sequence length
   int nq;               // n / 32
   int num_tiles;        // BH * ceil(nq / 4)

@@ -18,11 +18,11 @@ from ._lib import WiseShape, check, lib
 BLOCK = 32
 
 
-def shape_of(q: torch.Tensor, scale: float | None = None) -> WiseShape:
+def shape_of(q: torch.Tensor, scale: float | None = None, kv_heads: int = 0) -> WiseShape:
     if q.dim() != 4:
         raise ValueError("expected [batch, heads, seqlen, head_dim]")
     b, h, n, d = q.shape
-    return WiseShape(b, h, n, d, float(scale) if scale else 0.0)
+    return WiseShape(b, h, n, d, float(scale) if scale else 0.0, int(kv_heads))
 
 
 def _ptr(t: torch.Tensor | None) -> int | None:
@@ -34,13 +34,19 @@ def _stream(stream) -> int:
     return s.cuda_stream
 
 
-def _check_qkv(*ts: torch.Tensor) -> None:
-    ref = ts[0]
-    for t in ts:
+def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor) -> int:
+    """Validate q/o [B, H, n, d] and k/v [B, H_kv, n, d]; returns H_kv (grouped-query
+    attention when H_kv < H: query head h reads K/V head h // (H // H_kv))."""
+    for t in (q, k, v, o):
         if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
             raise ValueError("q/k/v/o must be contiguous bf16 CUDA tensors")
-        if t.shape != ref.shape:
-            raise ValueError("q/k/v/o shapes differ")
+    if o.shape != q.shape or v.shape != k.shape:
+        raise ValueError("o must match q and v must match k")
+    if q.dim() != 4 or k.dim() != 4 or k.shape[0] != q.shape[0] or k.shape[2:] != q.shape[2:]:
+        raise ValueError("k/v must be [batch, kv_heads, seqlen, head_dim] matching q")
+    if k.shape[1] < 1 or q.shape[1] % k.shape[1] != 0:
+        raise ValueError("query heads must be a multiple of k/v heads")
+    return int(k.shape[1])
 
 
 def words_per_row(nq: int) -> int:
@@ -58,7 +64,7 @@ def full_attn_mass(q, k, v, *, with_mass: bool = False, o=None, lse=None, mass=N
     b, h, n, d = q.shape
     if o is None:
         o = torch.empty_like(q)
-    _check_qkv(q, k, v, o)
+    kv = _check_qkv(q, k, v, o)
     if with_mass and mass is None:
         mass = torch.empty(b, h, n // BLOCK, n // BLOCK, dtype=torch.float32, device=q.device)
     if mass is not None and lse is None:
@@ -68,7 +74,7 @@ def full_attn_mass(q, k, v, *, with_mass: bool = False, o=None, lse=None, mass=N
     ws = workspace if (mass is not None and one_pass) else None
     rc = lib.wise_full_attn_mass(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(mass),
                                  _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
-                                 shape_of(q, scale), _stream(stream))
+                                 shape_of(q, scale, kv), _stream(stream))
     check(rc, "wise_full_attn_mass")
     return o, lse, mass
 
@@ -130,11 +136,11 @@ def sparse_attn(q, k, v, row_offsets, col_idx, col_count: int | None = None, *, 
     """Block-sparse causal attention over a CSR schedule.  Returns (o, lse)."""
     if o is None:
         o = torch.empty_like(q)
-    _check_qkv(q, k, v, o)
+    kv = _check_qkv(q, k, v, o)
     if col_count is None:
         col_count = col_idx.numel()
     rc = lib.wise_sparse_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(row_offsets),
-                              _ptr(col_idx), int(col_count), _ptr(lse), shape_of(q, scale),
+                              _ptr(col_idx), int(col_count), _ptr(lse), shape_of(q, scale, kv),
                               _stream(stream))
     check(rc, "wise_sparse_attn")
     return o, lse

@@ -57,6 +57,28 @@ def test_bad_shapes_rejected(lib, b, h, n, d):
     assert L.wise_schedule_max_nnz(shape(lib, b, h, n, d)) == -1
 
 
+def test_shape_struct_matches_header(lib):
+    """The ctypes mirror of wise_shape_t has the header's fields, in order."""
+    src = open(os.path.join(ROOT, "include", "wise.h")).read()
+    body = re.search(r"typedef struct wise_shape \{(.*?)\} wise_shape_t;", src, flags=re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = re.findall(r"(?:int32_t|float)\s+(\w+);", body)
+    assert fields == [f[0] for f in lib.WiseShape._fields_]
+    assert ctypes.sizeof(lib.WiseShape) == 4 * len(fields)
+
+
+@pytest.mark.parametrize("h,kv", [(6, 4), (8, 3), (4, -1)])
+def test_kv_heads_must_divide_heads(lib, h, kv):
+    L = lib.lib
+    fake = 1 << 20
+    s = lib.WiseShape(1, h, 256, 64, 0.0, kv)
+    assert L.wise_full_attn_mass(fake, fake, fake, fake, None, None, None, 0, s, None) == \
+        lib.WISE_ERR_SHAPE
+    assert "kv_heads" in lib.last_error()
+    assert L.wise_sparse_attn(fake, fake, fake, fake, fake, fake, 1, None, s, None) == \
+        lib.WISE_ERR_SHAPE
+
+
 def test_null_and_alignment_rejected(lib):
     L = lib.lib
     s = shape(lib)

@@ -98,6 +98,37 @@ def test_dense_many_tiles_per_cta(ops, b, h, n, d):
                 assert np.abs(np.tril(mass[bi, hi]) - O.block_mass(qf, kf)).max() <= MASS_TOL
 
 
+# Grouped-query attention: K/V carry fewer heads; query head h reads K/V head h // (H // H_kv).
+GQA_SHAPES = [(1, 8, 512, 128, 2), (2, 6, 256, 64, 3), (1, 32, 1024, 128, 8), (1, 4, 544, 96, 1)]
+
+
+@pytest.mark.parametrize("b,h,n,d,hkv", GQA_SHAPES)
+def test_gqa_dense_mass_and_sparse(ops, b, h, n, d, hkv):
+    g = h // hkv
+    nq = n // 32
+    qb, _, _ = rand_qkv_bits(b, h, n, d, seed=11 * n + h)
+    _, kb, vb = rand_qkv_bits(b, hkv, n, d, seed=13 * n + hkv)
+    q, k, v = to_dev(qb), to_dev(kb), to_dev(vb)
+    o, lse, mass = ops.full_attn_mass(q, k, v, with_mass=True)
+    rng = np.random.default_rng(n + h)
+    sups = [random_support(nq, rng, p=0.35) for _ in range(b * h)]
+    ro, ci, nnz = csr_device(sups)
+    o_s, _ = ops.sparse_attn(q, k, v, ro, ci, nnz)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    o, lse, mass, o_s = dev_f32(o), lse.cpu().numpy(), mass.cpu().numpy(), dev_f32(o_s)
+    for bi in range(b):
+        for hi in range(h):
+            qf = bf16_bits_to_f64(qb[bi, hi])
+            kf, vf = (bf16_bits_to_f64(x[bi, hi // g]) for x in (kb, vb))
+            o_ref, lse_ref = O.causal_attention(qf, kf, vf)
+            compare_o(o[bi, hi], o_ref, f"O[{bi},{hi}]")
+            assert np.abs(lse[bi, hi] - lse_ref).max() <= LSE_TOL
+            assert np.abs(np.tril(mass[bi, hi]) - O.block_mass(qf, kf)).max() <= MASS_TOL
+            os_ref, _ = O.masked_attention(qf, kf, vf, sups[bi * h + hi])
+            compare_o(o_s[bi, hi], os_ref, f"sparse O[{bi},{hi}]")
+
+
 def random_support(nq, rng, p=0.4, diag=True, empty_rows=()):
     s = np.tril(rng.random((nq, nq)) < p)
     if diag:
