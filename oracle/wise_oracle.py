@@ -79,28 +79,43 @@ def attention_probs(q, k, scale=None) -> np.ndarray:
     return p / p.sum(axis=1, keepdims=True)
 
 
-def block_mass(q, k, scale=None) -> np.ndarray:
+def block_mass(q, k, scale=None, block: int = BLOCK) -> np.ndarray:
     """Block-level attention mass r_qb (WISE paper §5.1, the block-mass equation).
 
-    r_qb = (1/|I_q|) * sum_{i in I_q} sum_{j in I_b} A_ij with B = 32 and A the
-    unrestricted causal softmax of the step.  Returns r [nq, nq]; entries with
-    b > q are exactly zero (no admissible key there).  Computed one query block
-    at a time (the definition is per query block).
+    r_qb = (1/|I_q|) * sum_{i in I_q} sum_{j in I_b} A_ij with blocks of ``block``
+    tokens (B = 32 unless a block-size variant of §7.3 is asked for) and A the
+    unrestricted causal softmax of the step.  Returns r [n/B, n/B]; entries with
+    b > q are exactly zero (no admissible key there).  Computed one query block at a
+    time (the definition is per query block).
     """
     q, k = np.asarray(q, np.float64), np.asarray(k, np.float64)
     n = q.shape[0]
-    assert n % BLOCK == 0
-    nq = n // BLOCK
+    assert n % block == 0
+    nb = n // block
     scale = default_scale(q.shape[1]) if scale is None else float(scale)
-    r = np.zeros((nq, nq))
-    for qb in range(nq):
-        rows = slice(qb * BLOCK, (qb + 1) * BLOCK)
+    r = np.zeros((nb, nb))
+    for qb in range(nb):
+        rows = slice(qb * block, (qb + 1) * block)
         s = _causal_scores(q, k, scale, rows)
         p = np.exp(s - s.max(axis=1, keepdims=True))
-        a = p / p.sum(axis=1, keepdims=True)              # rows of A for I_q
-        per_block = a.reshape(BLOCK, nq, BLOCK).sum(axis=2)  # sum over j in I_b
-        r[qb] = per_block.sum(axis=0) / BLOCK               # mean over i in I_q
+        a = p / p.sum(axis=1, keepdims=True)                 # rows of A for I_q
+        per_block = a.reshape(block, nb, block).sum(axis=2)  # sum over j in I_b
+        r[qb] = per_block.sum(axis=0) / block                # mean over i in I_q
     return r
+
+
+def expand_support(sel: np.ndarray, factor: int) -> np.ndarray:
+    """A support chosen on blocks of ``factor`` x 32 tokens, as 32 x 32 blocks.
+
+    The WISE paper runs its larger block sizes as exact 32 x 32 physical subtiles
+    (§7.3, the block-size study): query block q (of 32) of coarse block Q = q // factor
+    keeps key block b (of 32) iff its coarse block b // factor is in Q's support and
+    b <= q (the causal part of the coarse diagonal block).  ``sel`` is the coarse
+    [nQ, nQ] boolean support; returns the fine [nQ*factor, nQ*factor] one.
+    """
+    sel = np.asarray(sel, dtype=bool)
+    fine = np.repeat(np.repeat(sel, factor, axis=0), factor, axis=1)
+    return fine & np.tril(np.ones_like(fine))
 
 
 def eta_order(r_row: np.ndarray) -> np.ndarray:

@@ -169,6 +169,78 @@ def test_block_mass_equals_blocks_of_attention_matrix():
             assert abs(r[qb, b] - A[qb * B:(qb + 1) * B, b * B:(b + 1) * B].sum() / B) < 1e-13
 
 
+# --------------------------------------------------------------------------- block-size variants
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_block_mass_uniform_closed_form_larger_blocks(block):
+    """Q = 0 at B = 64 / 128: r_QB = mean_i |I_B cap [0, i]| / (i + 1), exact fractions."""
+    nb = 3
+    n = nb * block
+    _, k, _ = rand_qkv(n, 4, 18)
+    r = O.block_mass(np.zeros((n, 4)), k, block=block)
+    assert r.shape == (nb, nb)
+    for qb in range(nb):
+        for b in range(nb):
+            exact = Fraction(0)
+            for i in range(qb * block, (qb + 1) * block):
+                seen = max(0, min(i, (b + 1) * block - 1) - b * block + 1)
+                exact += Fraction(seen, i + 1)
+            exact /= block
+            assert abs(r[qb, b] - float(exact)) < 1e-14
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_block_mass_larger_blocks_pool_the_attention_matrix(block):
+    """Brute force: r_QB is the mean over the B query rows of the attention mass inside I_B."""
+    q, k, _ = rand_qkv(2 * block, 8, 19, scale_q=2.5)
+    A = O.attention_probs(q, k)
+    r = O.block_mass(q, k, block=block)
+    np.testing.assert_allclose(r.sum(axis=1), 1.0, atol=1e-12)
+    for qb in range(2):
+        for b in range(2):
+            ref = A[qb * block:(qb + 1) * block, b * block:(b + 1) * block].sum() / block
+            assert abs(r[qb, b] - ref) < 1e-13
+    assert r[0, 1] == 0.0
+
+
+def _element_mask_coarse(sel, factor, n):
+    """Element (i, j) is attended iff j <= i and coarse block (i // 32f, j // 32f) is kept."""
+    cb = B * factor
+    return [[j <= i and bool(sel[i // cb][j // cb]) for j in range(n)] for i in range(n)]
+
+
+def _element_mask_fine(fine, n):
+    """Element (i, j) is attended iff j <= i and fine 32 x 32 block (i // 32, j // 32) is kept."""
+    return [[j <= i and bool(fine[i // B][j // B]) for j in range(n)] for i in range(n)]
+
+
+@pytest.mark.parametrize("factor", [2, 4])
+def test_expand_support_is_the_same_element_mask(factor):
+    """Running a coarse support as 32 x 32 subtiles attends exactly the same (i, j) pairs."""
+    rng = np.random.default_rng(20 + factor)
+    nQ = 3
+    n = nQ * factor * B
+    for _ in range(4):
+        sel = np.tril(rng.random((nQ, nQ)) < 0.6)
+        np.fill_diagonal(sel, True)
+        fine = O.expand_support(sel, factor)
+        assert fine.shape == (nQ * factor, nQ * factor)
+        assert _element_mask_fine(fine, n) == _element_mask_coarse(sel, factor, n)
+
+
+def test_expand_support_is_causal_and_keeps_fine_diagonal():
+    sel = np.ones((4, 4), dtype=bool)
+    for factor in (1, 2, 4):
+        fine = O.expand_support(np.tril(sel), factor)
+        assert not np.any(np.triu(fine, 1))
+        assert np.all(np.diag(fine))
+        # Full coarse support -> every causal fine block, nothing else.
+        assert np.array_equal(fine, np.tril(np.ones_like(fine)))
+    # factor 1 is the identity on a lower-triangular support.
+    s = np.array([[1, 0, 0], [1, 1, 0], [0, 1, 1]], dtype=bool)
+    assert np.array_equal(O.expand_support(s, 1), s)
+
+
 # --------------------------------------------------------------------------- selection
 
 def test_eta_support_golden(golden_dir):
@@ -375,3 +447,23 @@ def test_pins_catch_planted_selection_mistakes(golden_dir):
         wrong = [c for c in g["cases"]
                  if mutant(np.array(c["r"]), c["eta"]).tolist() != c["support"]]
         assert wrong, mutant.__name__
+
+
+def _mutant_expand_no_causal_clip(sel, factor):
+    sel = np.asarray(sel, dtype=bool)
+    return np.repeat(np.repeat(sel, factor, axis=0), factor, axis=1)
+
+
+def _mutant_expand_transposed(sel, factor):
+    sel = np.asarray(sel, dtype=bool).T
+    fine = np.repeat(np.repeat(sel, factor, axis=0), factor, axis=1)
+    return fine & np.tril(np.ones_like(fine))
+
+
+def test_pins_catch_planted_expansion_mistakes():
+    """Dropping the causal clip leaves future fine blocks; transposing keeps the wrong ones."""
+    sel = np.array([[1, 0, 0], [1, 1, 0], [0, 1, 1]], dtype=bool)
+    factor, n = 2, 3 * 2 * B
+    want = _element_mask_coarse(sel, factor, n)
+    assert np.any(np.triu(_mutant_expand_no_causal_clip(sel, factor), 1))
+    assert _element_mask_fine(_mutant_expand_transposed(sel, factor), n) != want
