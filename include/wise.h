@@ -9,7 +9,8 @@
  *   exploration steps t <= t_d : wise_full_attn_mass   (dense causal attention,
  *                                  plus block mass on discovery-window steps)
  *                                wise_select_union     (cumulative-eta support,
- *                                  OR-ed into the working set)
+ *                                  OR-ed into the working set; or
+ *                                  wise_select_union_blocks for B = 64 / 128)
  *   once, after step t_d       : wise_build_schedule   (CSR key-block schedule)
  *   late steps t > t_d         : wise_sparse_attn      (block-sparse attention)
  *
@@ -122,6 +123,30 @@ size_t wise_mass_workspace_bytes(wise_shape_t shape);
  */
 int wise_select_union(const float* mass, uint32_t* union_bits, uint32_t* step_bits, float eta,
                       wise_shape_t shape, void* stream);
+
+/*
+ * Block-size variant of wise_select_union: the support is chosen on blocks of
+ * `block` tokens and run as exact 32 x 32 subtiles (WISE paper section 7.3, the
+ * block-size study).
+ *
+ * Defines: with F = block / 32, the mass of coarse block B for coarse query
+ * block Q is the block mass at block size 32F, R_QB = (1/F) sum over the F fine
+ * query blocks q of Q and the fine key blocks b <= q of B of mass[bh][q][b]
+ * (the block-mass equation of section 5.1 pooled exactly).  The coarse support
+ * is chosen as in wise_select_union (rank descending, ties to the lower coarse
+ * index, shortest prefix with cumulative mass >= eta, fp32 sums).  Fine row
+ * q = Q F + a then keeps fine block b iff coarse block b / F is kept and b <= q.
+ *
+ * mass, union_bits, step_bits, eta : as for wise_select_union; the bit masks
+ *              keep the fine [B, H, nq, W] layout, so wise_build_schedule and
+ *              wise_sparse_attn consume them unchanged.
+ * block      : 32, 64 or 128 tokens; 32 is exactly wise_select_union.
+ * Errors     : WISE_ERR_ARG (as wise_select_union, or another block size),
+ *              WISE_ERR_SHAPE (seqlen not a multiple of block, or as
+ *              wise_select_union), WISE_ERR_CUDA.
+ */
+int wise_select_union_blocks(const float* mass, uint32_t* union_bits, uint32_t* step_bits,
+                             float eta, int32_t block, wise_shape_t shape, void* stream);
 
 /* Workspace bytes wise_build_schedule needs for this shape (device memory). */
 size_t wise_schedule_workspace_bytes(wise_shape_t shape);

@@ -245,6 +245,25 @@ int wise_select_union(const float* mass, uint32_t* union_bits, uint32_t* step_bi
   return ok();
 }
 
+int wise_select_union_blocks(const float* mass, uint32_t* union_bits, uint32_t* step_bits,
+                             float eta, int32_t block, wise_shape_t shape, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!mass || !union_bits) return fail(WISE_ERR_ARG, "mass and union_bits must be non-NULL");
+  if (!(eta > 0.f)) return fail(WISE_ERR_ARG, "eta must be > 0 (got %g)", (double)eta);
+  if (block != 32 && block != 64 && block != 128)
+    return fail(WISE_ERR_ARG, "block must be 32, 64 or 128 (got %d)", (int)block);
+  if (shape.seqlen % block != 0)
+    return fail(WISE_ERR_SHAPE, "seqlen %d is not a multiple of block %d", (int)shape.seqlen,
+                (int)block);
+  const int nq = shape.seqlen / 32;
+  cudaError_t e = wise::launch_select_union_blocks(mass, union_bits, step_bits, eta, block / 32,
+                                                   shape.batch * shape.heads, nq,
+                                                   static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "select_union_blocks launch");
+  return ok();
+}
+
 size_t wise_schedule_workspace_bytes(wise_shape_t shape) {
   if (check_shape(shape)) return 0;
   const long long rows = (long long)shape.batch * shape.heads * (shape.seqlen / 32);

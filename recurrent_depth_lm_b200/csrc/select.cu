@@ -34,6 +34,42 @@ __device__ __forceinline__ float warp_sum_ge(const float (&v)[MAXW], const bool 
   return a;
 }
 
+// Shortest prefix of the (mass desc, index asc) ranking with cumulative mass >= eta,
+// for the masses v[s] of blocks s * 32 + lane that have ok[s] set.
+template <int MAXW>
+__device__ __forceinline__ void eta_cut(const float (&v)[MAXW], const bool (&ok)[MAXW], float eta,
+                                        int lane, bool (&sel)[MAXW]) {
+  const float total = warp_sum_ge<MAXW>(v, ok, 0.f);
+  if (!(eta < 1.0f) || total < eta) {
+#pragma unroll
+    for (int s = 0; s < MAXW; ++s) sel[s] = ok[s];
+    return;
+  }
+  // invariant: f(lo) >= eta, f(hi) < eta
+  uint32_t lo = 0u, hi = 0x7F800000u;
+  while (hi - lo > 1u) {
+    const uint32_t mid = lo + ((hi - lo) >> 1);
+    if (warp_sum_ge<MAXW>(v, ok, __uint_as_float(mid)) >= eta)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  const float tau = __uint_as_float(lo);
+  float running = warp_sum_ge<MAXW>(v, ok, __uint_as_float(hi));  // mass strictly above tau
+#pragma unroll
+  for (int s = 0; s < MAXW; ++s) sel[s] = ok[s] && v[s] > tau;
+#pragma unroll
+  for (int s = 0; s < MAXW; ++s) {
+    uint32_t ties = __ballot_sync(0xffffffffu, ok[s] && v[s] == tau);
+    while (ties != 0u && running < eta) {
+      const int b = __ffs(ties) - 1;
+      ties &= ties - 1u;
+      running += tau;
+      if (lane == b) sel[s] = true;
+    }
+  }
+}
+
 template <int MAXW>
 __global__ void __launch_bounds__(256)
     select_union_kernel(const float* __restrict__ mass, uint32_t* __restrict__ ubits,
@@ -55,35 +91,7 @@ __global__ void __launch_bounds__(256)
   }
 
   bool sel[MAXW];
-  const float total = warp_sum_ge<MAXW>(v, ok, 0.f);
-  if (!(eta < 1.0f) || total < eta) {
-#pragma unroll
-    for (int s = 0; s < MAXW; ++s) sel[s] = ok[s];
-  } else {
-    // invariant: f(lo) >= eta, f(hi) < eta
-    uint32_t lo = 0u, hi = 0x7F800000u;
-    while (hi - lo > 1u) {
-      const uint32_t mid = lo + ((hi - lo) >> 1);
-      if (warp_sum_ge<MAXW>(v, ok, __uint_as_float(mid)) >= eta)
-        lo = mid;
-      else
-        hi = mid;
-    }
-    const float tau = __uint_as_float(lo);
-    float running = warp_sum_ge<MAXW>(v, ok, __uint_as_float(hi));  // mass strictly above tau
-#pragma unroll
-    for (int s = 0; s < MAXW; ++s) sel[s] = ok[s] && v[s] > tau;
-#pragma unroll
-    for (int s = 0; s < MAXW; ++s) {
-      uint32_t ties = __ballot_sync(0xffffffffu, ok[s] && v[s] == tau);
-      while (ties != 0u && running < eta) {
-        const int b = __ffs(ties) - 1;
-        ties &= ties - 1u;
-        running += tau;
-        if (lane == b) sel[s] = true;
-      }
-    }
-  }
+  eta_cut<MAXW>(v, ok, eta, lane, sel);
 
   uint32_t word = 0u;
 #pragma unroll
@@ -95,6 +103,77 @@ __global__ void __launch_bounds__(256)
     const long long at = row * W + lane;
     if (sbits != nullptr) sbits[at] = word;
     ubits[at] |= word;
+  }
+}
+
+// Block-size variant (WISE paper section 7.3): selection on blocks of F x 32 tokens,
+// run as exact 32 x 32 subtiles.  One warp per coarse row (bh, Q).  The coarse mass
+// is the pooled fine mass, R_QB = (1/F) sum_{q in Q} sum_{b in B, b <= q} r_qb, which
+// is the block-mass definition at block size 32F.  After the cut, fine row
+// q = Q F + a keeps fine block b iff coarse block b / F was kept and b <= q.
+// Fine masks are written in the fine [nq, W] layout, so the schedule builder and the
+// sparse kernel run unchanged.
+template <int MAXWC, int F>
+__global__ void __launch_bounds__(256)
+    select_union_pooled_kernel(const float* __restrict__ mass, uint32_t* __restrict__ ubits,
+                               uint32_t* __restrict__ sbits, float eta, long long crows, int nq) {
+  const int lane = threadIdx.x & 31;
+  const long long crow = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (crow >= crows) return;  // warp-uniform
+  const int nQ = nq / F;
+  const long long bh = crow / nQ;
+  const int Q = (int)(crow % nQ);
+  const int Wc = (nQ + 31) >> 5;
+  const int W = (nq + 31) >> 5;
+  const float* mrow = mass + (bh * nq + (long long)Q * F) * nq;  // fine row Q F
+
+  float v[MAXWC];
+  bool ok[MAXWC];
+#pragma unroll
+  for (int s = 0; s < MAXWC; ++s) {
+    const int cb = s * 32 + lane;
+    ok[s] = (s < Wc) && (cb <= Q);
+    float acc = 0.f;
+    if (ok[s]) {
+#pragma unroll
+      for (int a = 0; a < F; ++a)
+#pragma unroll
+        for (int c = 0; c < F; ++c)
+          if (cb * F + c <= Q * F + a) acc += mrow[(long long)a * nq + cb * F + c];
+    }
+    v[s] = acc * (1.0f / F);
+  }
+
+  bool sel[MAXWC];
+  eta_cut<MAXWC>(v, ok, eta, lane, sel);
+
+  // Fine word w covers fine blocks 32w .. 32w+31 = coarse blocks 32w/F .. (32w+31)/F,
+  // all in coarse slot w / F; lane i's bit is the kept flag of coarse block (32w+i)/F.
+  uint32_t word = 0u;
+#pragma unroll
+  for (int w = 0; w < MAXWC * F; ++w) {
+    const int c = (32 * w + lane) / F;
+    const bool bit = __shfl_sync(0xffffffffu, (int)sel[w / F], c & 31) != 0;
+    const uint32_t m = __ballot_sync(0xffffffffu, bit);
+    if (lane == w) word = m;
+  }
+  if (lane < W) {
+#pragma unroll
+    for (int a = 0; a < F; ++a) {
+      const int q = Q * F + a;
+      const int first = 32 * lane;  // fine block of bit 0 of this word
+      uint32_t clip;
+      if (first > q)
+        clip = 0u;
+      else if (q - first >= 31)
+        clip = 0xffffffffu;
+      else
+        clip = (2u << (q - first)) - 1u;
+      const uint32_t out = word & clip;
+      const long long at = (bh * nq + q) * W + lane;
+      if (sbits != nullptr) sbits[at] = out;
+      ubits[at] |= out;
+    }
   }
 }
 
@@ -118,6 +197,43 @@ cudaError_t launch_select_union(const float* mass, uint32_t* union_bits, uint32_
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();
+}
+
+template <int F>
+static cudaError_t launch_pooled(const float* mass, uint32_t* union_bits, uint32_t* step_bits,
+                                 float eta, int BH, int nq, cudaStream_t stream) {
+  const int nQ = nq / F;
+  const long long crows = (long long)BH * nQ;
+  const int Wc = (nQ + 31) / 32;
+  const int warps_per_block = 8;
+  const unsigned grid = (unsigned)((crows + warps_per_block - 1) / warps_per_block);
+  const dim3 block(32 * warps_per_block);
+  if (Wc <= 1)
+    select_union_pooled_kernel<1, F><<<grid, block, 0, stream>>>(mass, union_bits, step_bits, eta,
+                                                                 crows, nq);
+  else if (Wc <= 2)
+    select_union_pooled_kernel<2, F><<<grid, block, 0, stream>>>(mass, union_bits, step_bits, eta,
+                                                                 crows, nq);
+  else if (Wc <= 4)
+    select_union_pooled_kernel<4, F><<<grid, block, 0, stream>>>(mass, union_bits, step_bits, eta,
+                                                                 crows, nq);
+  else if (Wc <= 8)
+    select_union_pooled_kernel<8, F><<<grid, block, 0, stream>>>(mass, union_bits, step_bits, eta,
+                                                                 crows, nq);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_union_blocks(const float* mass, uint32_t* union_bits,
+                                       uint32_t* step_bits, float eta, int factor, int BH, int nq,
+                                       cudaStream_t stream) {
+  if (factor == 1)
+    return launch_select_union(mass, union_bits, step_bits, eta, BH, nq, stream);
+  if (nq % factor != 0) return cudaErrorInvalidValue;
+  if (factor == 2) return launch_pooled<2>(mass, union_bits, step_bits, eta, BH, nq, stream);
+  if (factor == 4) return launch_pooled<4>(mass, union_bits, step_bits, eta, BH, nq, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace wise

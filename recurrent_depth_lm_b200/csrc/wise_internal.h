@@ -42,6 +42,12 @@ cudaError_t launch_mass_from_blse(const float* blse, const float* lse, float* ma
 cudaError_t launch_select_union(const float* mass, uint32_t* union_bits, uint32_t* step_bits,
                                 float eta, int BH, int nq, cudaStream_t stream);
 
+// Selection on blocks of factor x 32 tokens (factor 1, 2 or 4; nq % factor == 0),
+// written back as fine 32 x 32 masks in the [BH, nq, W] layout.
+cudaError_t launch_select_union_blocks(const float* mass, uint32_t* union_bits,
+                                       uint32_t* step_bits, float eta, int factor, int BH, int nq,
+                                       cudaStream_t stream);
+
 size_t schedule_workspace_bytes(long long rows);
 cudaError_t launch_build_schedule(const uint32_t* union_bits, int32_t* row_offsets,
                                   int32_t* col_idx, long long capacity, void* workspace,

@@ -85,15 +85,24 @@ def mass_workspace(b: int, h: int, n: int, head_dim: int, device) -> torch.Tenso
 
 
 def select_union(mass, union_bits, eta: float, *, step_bits=None, head_dim: int = 128,
-                 scale=None, stream=None):
-    """OR the cumulative-eta support of `mass` into `union_bits` (in place)."""
+                 scale=None, block: int = BLOCK, stream=None):
+    """OR the cumulative-eta support of `mass` into `union_bits` (in place).
+
+    ``block`` > 32 selects on blocks of that many tokens (64 or 128) and writes the
+    result as 32 x 32 subtiles; ``mass`` is always the 32-token block mass.
+    """
     b, h, nq, _ = mass.shape
     shp = WiseShape(b, h, nq * BLOCK, head_dim, float(scale) if scale else 0.0)
     if mass.dtype != torch.float32 or union_bits.dtype != torch.int32:
         raise ValueError("mass must be float32 and union_bits int32 (uint32 bit patterns)")
-    rc = lib.wise_select_union(_ptr(mass), _ptr(union_bits), _ptr(step_bits), float(eta), shp,
-                               _stream(stream))
-    check(rc, "wise_select_union")
+    if block == BLOCK:
+        rc = lib.wise_select_union(_ptr(mass), _ptr(union_bits), _ptr(step_bits), float(eta),
+                                   shp, _stream(stream))
+        check(rc, "wise_select_union")
+    else:
+        rc = lib.wise_select_union_blocks(_ptr(mass), _ptr(union_bits), _ptr(step_bits),
+                                          float(eta), int(block), shp, _stream(stream))
+        check(rc, "wise_select_union_blocks")
     return union_bits
 
 

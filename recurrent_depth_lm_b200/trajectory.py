@@ -6,6 +6,8 @@ t <= t_d run unrestricted (dense) causal attention; steps t_d-3 .. t_d also
 select each query block's cumulative-eta key-block support and union it;
 after step t_d the union is compacted once into a CSR schedule; every later
 step runs block-sparse attention over that schedule with fresh Q, K, V.
+Section 7.3's block-size variants (block = 64 or 128) select on coarser blocks
+and run the result as exact 32 x 32 subtiles.
 
 All buffers are allocated once here with torch; the library calls only
 enqueue kernels on the current stream (no host synchronisation inside a
@@ -22,9 +24,12 @@ from . import ops
 class WiseTrajectory:
     def __init__(self, batch: int, heads: int, seqlen: int, head_dim: int, *, t_d: int = 12,
                  window=(9, 12), eta: float = 0.95, scale: float | None = None,
-                 device="cuda", keep_step_bits: bool = False):
-        if seqlen % ops.BLOCK:
-            raise ValueError("seqlen must be a multiple of 32")
+                 block: int = ops.BLOCK, device="cuda", keep_step_bits: bool = False):
+        if block not in (32, 64, 128):
+            raise ValueError("block must be 32, 64 or 128")
+        if seqlen % block:
+            raise ValueError(f"seqlen must be a multiple of the block size {block}")
+        self.block = block
         self.b, self.h, self.n, self.d = batch, heads, seqlen, head_dim
         self.nq = seqlen // ops.BLOCK
         self.t_d, self.window, self.eta = t_d, tuple(window), float(eta)
@@ -63,7 +68,8 @@ class WiseTrajectory:
                     sb = torch.empty_like(self.union)
                     self.step_bits[t] = sb
                 ops.select_union(self.mass, self.union, self.eta, step_bits=sb,
-                                 head_dim=self.d, scale=self.scale, stream=stream)
+                                 head_dim=self.d, scale=self.scale, block=self.block,
+                                 stream=stream)
             else:
                 o, _, _ = ops.full_attn_mass(q, k, v, o=o, lse=lse, scale=self.scale,
                                              stream=stream)

@@ -81,3 +81,22 @@ def check_csr(row_offsets: np.ndarray, col_idx: np.ndarray, support: np.ndarray)
 
 def head_f64(bits: np.ndarray) -> np.ndarray:
     return bf16_bits_to_f64(bits)
+
+
+def pool_mass(r: np.ndarray, factor: int) -> np.ndarray:
+    """[..., nq, nq] 32-token block masses -> [..., nq/f, nq/f] masses of f x 32-token blocks.
+
+    R_QB = (1/f) sum of r_qb over the f x f fine blocks (q in Q, b in B) with b <= q.
+    The oracle pins check this against the block mass computed at the larger size.
+    """
+    r = np.asarray(r, np.float64)
+    nq = r.shape[-1]
+    r = r * np.tril(np.ones((nq, nq)))
+    nQ = nq // factor
+    shp = r.shape[:-2] + (nQ, factor, nQ, factor)
+    return r.reshape(shp).sum(axis=(-3, -1)) / factor
+
+
+def coarse_of_fine(fine: np.ndarray, factor: int) -> np.ndarray:
+    """Coarse support read back from an expanded fine one: fine row Q f + f - 1, block B f."""
+    return fine[..., factor - 1::factor, ::factor]

@@ -98,6 +98,23 @@ def test_null_and_alignment_rejected(lib):
     assert "eta" in lib.last_error()
 
 
+
+def test_select_blocks_checks(lib):
+    L = lib.lib
+    s = shape(lib)
+    fake = 1 << 20
+    assert L.wise_select_union_blocks(None, fake, None, 0.95, 64, s, None) == lib.WISE_ERR_ARG
+    assert L.wise_select_union_blocks(fake, fake, None, -1.0, 64, s, None) == lib.WISE_ERR_ARG
+    for bad in (0, 16, 48, 96, 256):
+        assert L.wise_select_union_blocks(fake, fake, None, 0.95, bad, s, None) == \
+            lib.WISE_ERR_ARG
+        assert "block" in lib.last_error()
+    odd = lib.WiseShape(1, 2, 96, 64, 0.0, 0)       # 3 blocks of 32: not a multiple of 64
+    assert L.wise_select_union_blocks(fake, fake, None, 0.95, 64, odd, None) == lib.WISE_ERR_SHAPE
+    odd = lib.WiseShape(1, 2, 192, 64, 0.0, 0)      # 6 blocks of 32: not a multiple of 128
+    assert L.wise_select_union_blocks(fake, fake, None, 0.95, 128, odd, None) == \
+        lib.WISE_ERR_SHAPE
+
 def test_schedule_sizes_and_checks(lib):
     L = lib.lib
     s = shape(lib, 1, 32, 4096, 128)

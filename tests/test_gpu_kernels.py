@@ -8,8 +8,8 @@ import numpy as np
 import pytest
 
 from oracle import wise_oracle as O
-from parity_utils import (LSE_TOL, MASS_TOL, bits_to_bool, check_csr, compare_o,
-                          compare_selection)
+from parity_utils import (LSE_TOL, MASS_TOL, bits_to_bool, check_csr, coarse_of_fine, compare_o,
+                          compare_selection, pool_mass)
 from wise_inputs import bf16_bits_to_f64, f32_to_bf16_bits
 
 pytestmark = pytest.mark.gpu
@@ -345,6 +345,95 @@ def test_select_golden_ties_and_exact_cut(ops):
         u = bits_to_bool(union.cpu().numpy()[0, 0], nq)
         assert np.nonzero(u[nq - 1])[0].tolist() == c["support"], c["why"]
 
+
+
+def _peaky_masses(rng, bh, nq):
+    masses = np.zeros((bh, nq, nq))
+    for x in range(bh):
+        for q in range(nq):
+            lg = rng.standard_normal(q + 1) * 2.5
+            p = np.exp(lg - lg.max())
+            masses[x, q, : q + 1] = p / p.sum()
+    return masses
+
+
+def _check_blocks_selection(sel_fine, m_fine, f, eta):
+    """Fine support of one head: exactly the expansion of a coarse support, and that coarse
+    support is the oracle's selection on the pooled masses (near-cut rows exempt)."""
+    coarse = coarse_of_fine(sel_fine, f)
+    assert np.array_equal(sel_fine, O.expand_support(coarse, f))
+    R = pool_mass(np.tril(m_fine), f)
+    exempt = compare_selection(coarse, R, eta)
+    for Q in range(R.shape[0]):   # a row whose total is below eta keeps everything
+        assert R[Q][coarse[Q]].sum() >= min(eta, R[Q, : Q + 1].sum()) - 1e-6
+    return exempt
+
+
+@pytest.mark.parametrize("block", [64, 128])
+@pytest.mark.parametrize("nq,bh", [(8, 2), (40, 3), (128, 2), (512, 1)])
+def test_select_union_blocks_matches_oracle(ops, block, nq, bh):
+    """Block-size variant: selection on 64 / 128-token blocks, written as 32 x 32 subtiles."""
+    f = block // 32
+    rng = np.random.default_rng(nq * 5 + f)
+    eta = 0.95
+    m32 = _peaky_masses(rng, bh, nq).astype(np.float32)
+    garbage = m32.copy()
+    garbage[:, np.triu_indices(nq, 1)[0], np.triu_indices(nq, 1)[1]] = np.nan  # b > q: not read
+    union = ops.new_bitmask(1, bh, nq, "cuda")
+    step = torch.empty_like(union)
+    ops.select_union(torch.from_numpy(garbage).reshape(1, bh, nq, nq).cuda(), union, eta,
+                     step_bits=step, block=block)
+    m2 = np.roll(m32, 1, axis=2) * np.tril(np.ones((nq, nq), np.float32))
+    m2 /= np.maximum(m2.sum(axis=2, keepdims=True), 1e-30)
+    step2 = torch.empty_like(union)
+    ops.select_union(torch.from_numpy(m2).reshape(1, bh, nq, nq).cuda(), union, eta,
+                     step_bits=step2, block=block)
+    torch.cuda.synchronize()
+    s1 = bits_to_bool(step.cpu().numpy()[0], nq)
+    s2 = bits_to_bool(step2.cpu().numpy()[0], nq)
+    u = bits_to_bool(union.cpu().numpy()[0], nq)
+    assert np.array_equal(u, s1 | s2)
+    exempt = 0
+    for x in range(bh):
+        exempt += _check_blocks_selection(s1[x], m32[x].astype(np.float64), f, eta)
+        exempt += _check_blocks_selection(s2[x], m2[x].astype(np.float64), f, eta)
+    assert exempt <= 2
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_select_union_blocks_real_masses(ops, block):
+    """Fine masses of a real causal softmax; the reference is the oracle's block mass computed
+    directly at the larger block size (not pooled)."""
+    f = block // 32
+    n, d, eta = 1280, 16, 0.9
+    rng = np.random.default_rng(block)
+    q = rng.standard_normal((n, d)) * 2.0
+    k = rng.standard_normal((n, d))
+    r32 = O.block_mass(q, k).astype(np.float32)
+    nq = n // 32
+    union = ops.new_bitmask(1, 1, nq, "cuda")
+    ops.select_union(torch.from_numpy(r32).reshape(1, 1, nq, nq).cuda(), union, eta, block=block)
+    fine = bits_to_bool(union.cpu().numpy()[0, 0], nq)
+    coarse = coarse_of_fine(fine, f)
+    assert np.array_equal(fine, O.expand_support(coarse, f))
+    assert compare_selection(coarse, O.block_mass(q, k, block=block), eta) <= 1
+
+
+def test_select_union_blocks_32_is_the_plain_selection(ops):
+    """block = 32 through the variant entry point is exactly wise_select_union."""
+    nq, bh = 45, 2
+    m = _peaky_masses(np.random.default_rng(3), bh, nq).astype(np.float32)
+    dm = torch.from_numpy(m).reshape(1, bh, nq, nq).cuda()
+    a = ops.new_bitmask(1, bh, nq, "cuda")
+    b = ops.new_bitmask(1, bh, nq, "cuda")
+    ops.select_union(dm, a, 0.95)
+    from recurrent_depth_lm_b200._lib import lib, check
+    shp = ops.shape_of(torch.empty(1, bh, nq * 32, 128, dtype=torch.bfloat16, device="meta"))
+    check(lib.wise_select_union_blocks(dm.data_ptr(), b.data_ptr(), None, 0.95, 32, shp,
+                                       torch.cuda.current_stream().cuda_stream),
+          "wise_select_union_blocks")
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
 
 @pytest.mark.parametrize("nq,bh", [(1, 1), (8, 2), (45, 3), (512, 2)])
 def test_build_schedule_bit_exact(ops, nq, bh):

@@ -7,7 +7,8 @@ dense O, block masses and per-step selections on window steps (bit-exact up to
 near-cut rows), union = OR of the step selections, schedule = CSR of the union
 (bit-exact), and late-step O against masked attention with the GPU's schedule.
 The 16K config also runs an eta = 1.0 trajectory whose late steps must equal
-dense causal attention.
+dense causal attention; the 1K config also runs the 64 / 128-token block-size
+variants (selection on the coarse masses, run as 32 x 32 subtiles).
 """
 
 import os
@@ -16,7 +17,8 @@ import numpy as np
 import pytest
 
 from oracle import wise_oracle as O
-from parity_utils import (MASS_TOL, bits_to_bool, check_csr, compare_o, compare_selection)
+from parity_utils import (MASS_TOL, bits_to_bool, check_csr, coarse_of_fine, compare_o,
+                          compare_selection)
 from wise_inputs import CONFIGS, bf16_bits_to_f64, iter_steps
 from wise_inputs.generator import StepPool
 
@@ -28,7 +30,7 @@ def _dev(bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
 
 
-def run_config(cfg, sample, check_steps, etas=(None,)):
+def run_config(cfg, sample, check_steps, etas=(None,), block=32):
     """Run all heads of `cfg` on the GPU; return host copies for the sampled heads."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
@@ -36,7 +38,7 @@ def run_config(cfg, sample, check_steps, etas=(None,)):
     idx = [b * cfg.heads + h for (b, h) in sample]
     trajs = {eta: WiseTrajectory(cfg.batch, cfg.heads, cfg.seqlen, cfg.head_dim, t_d=cfg.t_d,
                                  window=cfg.window, eta=cfg.eta if eta is None else eta,
-                                 keep_step_bits=True) for eta in etas}
+                                 block=block, keep_step_bits=True) for eta in etas}
     res = {eta: {"o": {}, "mass": {}, "bits": {}} for eta in etas}
     workers = max(1, min(16, (os.cpu_count() or 2)))
     with StepPool(cfg, workers=workers) as pool:
@@ -63,8 +65,9 @@ def run_config(cfg, sample, check_steps, etas=(None,)):
     return res
 
 
-def check_config(cfg, sample, check_steps, etas=(None,)):
-    res = run_config(cfg, sample, check_steps, etas)
+def check_config(cfg, sample, check_steps, etas=(None,), block=32):
+    res = run_config(cfg, sample, check_steps, etas, block)
+    f = block // 32
     nq = cfg.nq
     host = {t: (q, k, v) for t, q, k, v in iter_steps(cfg, heads=sample)}
     report = {}
@@ -80,7 +83,12 @@ def check_config(cfg, sample, check_steps, etas=(None,)):
                 r_ref = O.block_mass(q, k, cfg.scale)
                 assert np.abs(np.tril(r["mass"][t][si]) - r_ref).max() <= MASS_TOL
                 sel_gpu = bits_to_bool(r["bits"][t][si], nq)
-                exempt += compare_selection(sel_gpu, r_ref, e)
+                if f == 1:
+                    exempt += compare_selection(sel_gpu, r_ref, e)
+                else:   # block-size variant: coarse selection, run as 32 x 32 subtiles
+                    coarse = coarse_of_fine(sel_gpu, f)
+                    assert np.array_equal(sel_gpu, O.expand_support(coarse, f))
+                    exempt += compare_selection(coarse, O.block_mass(q, k, cfg.scale, block), e)
                 step_sel.append(sel_gpu)
             union = bits_to_bool(r["union"][si], nq)
             assert np.array_equal(union, O.temporal_union(step_sel))
@@ -110,6 +118,13 @@ def test_trajectory_tiny_all_heads_all_steps():
 def test_trajectory_1k():
     cfg = CONFIGS["1k"]
     check_config(cfg, [(0, 0), (0, 13), (0, 31)], check_steps=range(1, cfg.steps + 1))
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_trajectory_1k_block_sizes(block):
+    cfg = CONFIGS["1k"]
+    rep = check_config(cfg, [(0, 0), (0, 31)], check_steps=[12, 13, 32], block=block)
+    assert rep[None]["exempt_rows"] <= 2
 
 
 def test_trajectory_4k():

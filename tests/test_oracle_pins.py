@@ -203,6 +203,16 @@ def test_block_mass_larger_blocks_pool_the_attention_matrix(block):
     assert r[0, 1] == 0.0
 
 
+
+@pytest.mark.parametrize("factor", [2, 4])
+def test_pooled_fine_mass_is_block_mass_at_larger_size(factor):
+    """The identity the GPU selection relies on: pooling 32-token masses gives B = 32f masses."""
+    from parity_utils import pool_mass
+    q, k, _ = rand_qkv(3 * factor * B, 8, 21, scale_q=2.0)
+    r = O.block_mass(q, k)
+    np.testing.assert_allclose(pool_mass(r, factor), O.block_mass(q, k, block=B * factor),
+                               atol=1e-13, rtol=0)
+
 def _element_mask_coarse(sel, factor, n):
     """Element (i, j) is attended iff j <= i and coarse block (i // 32f, j // 32f) is kept."""
     cb = B * factor
