@@ -12,9 +12,11 @@ admissible (query, key) pair of the dense steps and of the selected blocks of
 the late steps (the mass pass recompute and masked work are not counted).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4k]
-       [--impl wise|reference].  For N > 1 launch one process per GPU with
-torch.distributed.run; every rank runs its own independent trajectory
-(weak scaling, no collective on the data path).
+       [--block 32|64|128] [--impl wise|reference].  --block selects on
+coarser blocks (appendix C.6's block-size study) and runs them as 32 x 32
+subtiles.  For N > 1 launch one process per GPU with torch.distributed.run;
+every rank runs its own independent trajectory (weak scaling, no collective
+on the data path).
 """
 
 from __future__ import annotations
@@ -209,13 +211,13 @@ def make_inputs(cfg, rank: int, device, workers: int):
 class TrajectoryRunner:
     """Runs whole trajectories through the C ABI with per-call CUDA events."""
 
-    def __init__(self, cfg, device):
+    def __init__(self, cfg, device, block: int = 32):
         import torch
         from recurrent_depth_lm_b200 import ops
         from recurrent_depth_lm_b200.trajectory import WiseTrajectory
-        self.cfg, self.ops = cfg, ops
+        self.cfg, self.ops, self.block = cfg, ops, block
         self.traj = WiseTrajectory(cfg.batch, cfg.heads, cfg.seqlen, cfg.head_dim, t_d=cfg.t_d,
-                                   window=cfg.window, eta=cfg.eta, device=device)
+                                   window=cfg.window, eta=cfg.eta, block=block, device=device)
         self.o = torch.empty(cfg.batch, cfg.heads, cfg.seqlen, cfg.head_dim,
                              dtype=torch.bfloat16, device=device)
         self.device = device
@@ -245,7 +247,8 @@ class TrajectoryRunner:
                     ops.full_attn_mass(qt, kt, vt, o=self.o, lse=tr.lse, mass=tr.mass,
                                        workspace=tr.mass_ws)
                     b = ev() if events is not None else None
-                    ops.select_union(tr.mass, tr.union, cfg.eta, head_dim=cfg.head_dim)
+                    ops.select_union(tr.mass, tr.union, cfg.eta, head_dim=cfg.head_dim,
+                                     block=self.block)
                     c = ev() if events is not None else None
                     if events is not None:
                         events.setdefault("dense_mass", []).append((a, b))
@@ -322,7 +325,7 @@ def run_e2e(cfg, runner, host_q, host_k, host_v, reps: int):
     return dt, 3 * T * per, T * per
 
 
-def cpu_oracle_sample(cfg, n_heads: int = 1):
+def cpu_oracle_sample(cfg, n_heads: int = 1, block: int = 32):
     """The CPU oracle, as it stands, on a bounded sample: for each sampled head one
     exploration step (dense attention + block mass + eta-selection -> schedule) and
     one late block-sparse step.  Returns (seconds, useful FLOPs, description)."""
@@ -339,8 +342,10 @@ def cpu_oracle_sample(cfg, n_heads: int = 1):
     for i in range(len(heads)):
         q, k, v = (bf16_bits_to_f64(x[i]) for x in steps[cfg.t_d])
         O.causal_attention(q, k, v, cfg.scale)
-        r = O.block_mass(q, k, cfg.scale)
+        r = O.block_mass(q, k, cfg.scale, block=block)
         sup = O.select(r, cfg.eta)
+        if block != 32:
+            sup = O.expand_support(sup, block // 32)
         ro, ci = O.csr_schedule(sup)
         q, k, v = (bf16_bits_to_f64(x[i]) for x in steps[cfg.t_d + 1])
         O.sparse_attention(q, k, v, ro, ci, cfg.scale)
@@ -349,7 +354,7 @@ def cpu_oracle_sample(cfg, n_heads: int = 1):
         flops += sparse_flops(cfg.with_(batch=1, heads=1), ro, ci)
     dt = time.perf_counter() - t0
     desc = (f"{len(heads)} head(s) of {cfg.name}: one dense exploration step with block mass and "
-            f"eta-selection, plus one block-sparse late step, numpy float64")
+            f"eta-selection (B={block}), plus one block-sparse late step, numpy float64")
     return dt, flops, desc
 
 
@@ -375,7 +380,7 @@ def bench_wise(args):
     workers = args.workers or max(1, min(16, (os.cpu_count() or 2) // max(1, world)))
 
     q, k, v, _ = make_inputs(cfg, rank, device, workers)
-    runner = TrajectoryRunner(cfg, device)
+    runner = TrajectoryRunner(cfg, device, block=args.block)
     ops = runner.ops
 
     for _ in range(args.warmup):
@@ -450,7 +455,7 @@ def bench_wise(args):
 
     cpu = None
     if rank == 0 and world == 1 and args.cpu_baseline:
-        secs, fl, desc = cpu_oracle_sample(cfg, n_heads=args.cpu_heads)
+        secs, fl, desc = cpu_oracle_sample(cfg, n_heads=args.cpu_heads, block=args.block)
         cpu = {"value": round(fl / secs / 1e12, 6), "unit": UNIT, "cores": blas_threads(),
                "kind": "oracle", "sample": desc, "seconds": round(secs, 2)}
 
@@ -461,7 +466,9 @@ def bench_wise(args):
         "data": "synthetic (seeded generator standing in for the pages' saved Huginn workloads)",
         "config": {"workload": f"{cfg.name}: batch {cfg.batch}, {cfg.heads} heads, head_dim "
                                f"{cfg.head_dim}, n={cfg.seqlen}, T={cfg.steps}, dense 1-{cfg.t_d}, "
-                               f"union {cfg.window[0]}-{cfg.window[1]}, eta={cfg.eta}, B=32",
+                               f"union {cfg.window[0]}-{cfg.window[1]}, eta={cfg.eta}, "
+                               f"B={args.block}"
+                               + (" (run as 32x32 subtiles)" if args.block != 32 else ""),
                    "step": "one full WISE trajectory (dense + mass/select + schedule + sparse)",
                    "l2": "inputs larger than L2: every trajectory streams "
                          f"{3 * cfg.steps * cfg.bh * cfg.seqlen * cfg.head_dim * 2 / 1e9:.2f} GB "
@@ -499,11 +506,11 @@ def bench_reference(args):
     from wise_inputs import CONFIGS
     cfg = CONFIGS[args.config]
     for _ in range(args.warmup):
-        cpu_oracle_sample(cfg, n_heads=1)
+        cpu_oracle_sample(cfg, n_heads=1, block=args.block)
     secs, flops = 0.0, 0.0
     desc = ""
     for _ in range(args.steps):
-        s, f, desc = cpu_oracle_sample(cfg, n_heads=1)
+        s, f, desc = cpu_oracle_sample(cfg, n_heads=1, block=args.block)
         secs += s
         flops += f
     value = flops / secs / 1e12
@@ -513,7 +520,8 @@ def bench_reference(args):
         "ms_per_step": round(secs / args.steps * 1e3, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "impl": "reference",
         "data": "synthetic (seeded generator)",
-        "config": {"workload": cfg.name, "step": "bounded oracle sample (see cpu_baseline)"},
+        "config": {"workload": f"{cfg.name}, B={args.block}",
+                   "step": "bounded oracle sample (see cpu_baseline)"},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "kind": "oracle",
                          "cores": blas_threads(), "sample": desc},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -529,6 +537,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["wise", "reference"], default="wise")
     ap.add_argument("--config", default="4k")
+    ap.add_argument("--block", type=int, choices=[32, 64, 128], default=32,
+                    help="selection block size (64 / 128 run as 32x32 subtiles)")
     ap.add_argument("--workers", type=int, default=0)
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--e2e-reps", type=int, default=2)

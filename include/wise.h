@@ -126,8 +126,8 @@ int wise_select_union(const float* mass, uint32_t* union_bits, uint32_t* step_bi
 
 /*
  * Block-size variant of wise_select_union: the support is chosen on blocks of
- * `block` tokens and run as exact 32 x 32 subtiles (WISE paper section 7.3, the
- * block-size study).
+ * `block` tokens and run as exact 32 x 32 subtiles (WISE paper appendix C.6,
+ * "Block-Size Tradeoff").
  *
  * Defines: with F = block / 32, the mass of coarse block B for coarse query
  * block Q is the block mass at block size 32F, R_QB = (1/F) sum over the F fine

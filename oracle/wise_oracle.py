@@ -83,7 +83,7 @@ def block_mass(q, k, scale=None, block: int = BLOCK) -> np.ndarray:
     """Block-level attention mass r_qb (WISE paper §5.1, the block-mass equation).
 
     r_qb = (1/|I_q|) * sum_{i in I_q} sum_{j in I_b} A_ij with blocks of ``block``
-    tokens (B = 32 unless a block-size variant of §7.3 is asked for) and A the
+    tokens (B = 32 unless a block-size variant of App. C.6 is asked for) and A the
     unrestricted causal softmax of the step.  Returns r [n/B, n/B]; entries with
     b > q are exactly zero (no admissible key there).  Computed one query block at a
     time (the definition is per query block).
@@ -108,7 +108,7 @@ def expand_support(sel: np.ndarray, factor: int) -> np.ndarray:
     """A support chosen on blocks of ``factor`` x 32 tokens, as 32 x 32 blocks.
 
     The WISE paper runs its larger block sizes as exact 32 x 32 physical subtiles
-    (§7.3, the block-size study): query block q (of 32) of coarse block Q = q // factor
+    (App. C.6, "Block-Size Tradeoff"): query block q (of 32) of coarse block Q = q // factor
     keeps key block b (of 32) iff its coarse block b // factor is in Q's support and
     b <= q (the causal part of the coarse diagonal block).  ``sel`` is the coarse
     [nQ, nQ] boolean support; returns the fine [nQ*factor, nQ*factor] one.

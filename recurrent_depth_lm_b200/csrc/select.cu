@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Block-size variant (WISE paper section 7.3): selection on blocks of F x 32 tokens,
+// Block-size variant (WISE paper appendix C.6, "Block-Size Tradeoff"): selection on blocks of F x 32 tokens,
 // run as exact 32 x 32 subtiles.  One warp per coarse row (bh, Q).  The coarse mass
 // is the pooled fine mass, R_QB = (1/F) sum_{q in Q} sum_{b in B, b <= q} r_qb, which
 // is the block-mass definition at block size 32F.  After the cut, fine row

@@ -6,7 +6,7 @@ t <= t_d run unrestricted (dense) causal attention; steps t_d-3 .. t_d also
 select each query block's cumulative-eta key-block support and union it;
 after step t_d the union is compacted once into a CSR schedule; every later
 step runs block-sparse attention over that schedule with fresh Q, K, V.
-Section 7.3's block-size variants (block = 64 or 128) select on coarser blocks
+Appendix C.6's block-size variants (block = 64 or 128) select on coarser blocks
 and run the result as exact 32 x 32 subtiles.
 
 All buffers are allocated once here with torch; the library calls only
