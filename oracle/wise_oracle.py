@@ -28,6 +28,8 @@ Readings of points the paper leaves open (also listed in the design notes):
 
 from __future__ import annotations
 
+import math
+
 import numpy as np
 
 BLOCK = 32
@@ -234,6 +236,61 @@ def block_density(support: np.ndarray) -> float:
     """Fraction of admissible (causal) query-key blocks retained (App. B, evaluation metrics)."""
     nq = support.shape[0]
     return float(np.tril(support).sum()) / (nq * (nq + 1) / 2)
+
+
+def retained_mass(r: np.ndarray, support: np.ndarray) -> np.ndarray:
+    """Share of one step's unrestricted attention mass that falls inside a support.
+
+    WISE paper App. B, "Evaluation metrics": retained (future) attention mass is the
+    fraction of the unrestricted Full-attention mass that lies inside the frozen
+    support.  Per query block q this is sum over kept admissible blocks b <= q of
+    r_qb (the block mass of that step, §5.1), which is the mean over the rows i of q
+    of sum_{j : b(j) kept} A_ij.  Returns [nq]; the mean over query blocks is the
+    per-token average, since every block has 32 rows.  Sums are correctly rounded
+    (math.fsum), so they do not depend on summation order.
+    """
+    r = np.asarray(r, np.float64)
+    keep = np.tril(np.asarray(support, dtype=bool))
+    return np.array([math.fsum(r[qb][keep[qb]]) for qb in range(r.shape[0])])
+
+
+def static_support(r1: np.ndarray, eta: float = 0.95) -> np.ndarray:
+    """Static-95 control (App. B, "Intervention controls"): the cumulative-eta
+    support of the FIRST recurrent step alone, S_q = B_q^(1, 0.95)."""
+    return select(r1, eta)
+
+
+def size_matched(r1: np.ndarray, ref: np.ndarray) -> np.ndarray:
+    """SizeMatched control (App. B, "Intervention controls"): per query block, the
+    K_q admissible blocks of largest step-1 mass, K_q = |W_q| the size of the
+    reference (WISE) working set row; TopK ties go to the lower block index."""
+    nq = r1.shape[0]
+    ref = np.tril(np.asarray(ref, dtype=bool))
+    sel = np.zeros((nq, nq), dtype=bool)
+    for qb in range(nq):
+        k = int(ref[qb].sum())
+        sel[qb, eta_order(r1[qb, : qb + 1])[:k]] = True
+    return sel
+
+
+def mass_matched(r1: np.ndarray, ref: np.ndarray) -> np.ndarray:
+    """MassMatched control (App. B, "Intervention controls"): m_q = sum over the
+    reference (WISE) working set W_q of the step-1 block masses, and the control keeps
+    the fewest step-1-ranked blocks (mass descending, ties to the lower index) whose
+    step-1 mass reaches m_q: the cumulative-eta support of step 1 at eta = m_q.
+    m_q and every prefix sum are correctly rounded (math.fsum), so a prefix holding
+    the same blocks as W_q reaches m_q exactly; an empty W_q gives an empty row.
+    """
+    r1 = np.asarray(r1, np.float64)
+    nq = r1.shape[0]
+    m = retained_mass(r1, ref)
+    sel = np.zeros((nq, nq), dtype=bool)
+    for qb in range(nq):
+        row = r1[qb, : qb + 1]
+        order = eta_order(row)
+        k = next((k for k in range(qb + 2) if math.fsum(row[order[:k]]) >= m[qb]), qb + 1)
+        sel[qb, order[:k]] = True
+    return sel
 
 
 def head_trajectory(steps, t_d: int, window, eta: float, scale=None, keep_dense_o=True):

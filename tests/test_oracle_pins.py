@@ -400,6 +400,129 @@ def test_tiny_trajectory_structure():
     assert 0 < O.block_density(U) <= 1
 
 
+
+# --------------------------------------------------------------------------- controls and retained mass
+
+def test_retained_mass_brute_force():
+    """Retained mass of a support = mean over the rows of each query block of the attention
+    probability that falls on kept key blocks (scalar loops on a tiny case)."""
+    q, k, _ = rand_qkv(128, 3, 30, scale_q=2.0)
+    nq, scale = 4, 1 / math.sqrt(3)
+    rng = np.random.default_rng(30)
+    sup = rng.random((nq, nq)) < 0.5
+    ql, kl = q.tolist(), k.tolist()
+    want = []
+    for qb in range(nq):
+        tot = 0.0
+        for i in range(qb * B, (qb + 1) * B):
+            logits = [sum(ql[i][c] * kl[j][c] for c in range(3)) * scale for j in range(i + 1)]
+            mx = max(logits)
+            w = [math.exp(x - mx) for x in logits]
+            z = sum(w)
+            tot += sum(w[j] for j in range(i + 1) if sup[qb][j // B]) / z
+        want.append(tot / B)
+    got = O.retained_mass(O.block_mass(q, k), sup)
+    np.testing.assert_allclose(got, want, atol=1e-13, rtol=0)
+
+
+def test_retained_mass_special_supports():
+    q, k, _ = rand_qkv(256, 16, 31, scale_q=2.5)
+    r = O.block_mass(q, k)
+    nq = 8
+    np.testing.assert_allclose(O.retained_mass(r, np.ones((nq, nq), bool)), 1.0, atol=1e-12)
+    assert np.all(O.retained_mass(r, np.zeros((nq, nq), bool)) == 0.0)
+    assert np.all(O.retained_mass(r, O.select(r, 0.9)) >= 0.9)
+    # blocks above the diagonal carry no mass and are ignored even if set
+    assert np.array_equal(O.retained_mass(r, np.triu(np.ones((nq, nq), bool), 1)), np.zeros(nq))
+
+
+def _softmax_rows(rng, nq, temp=2.5):
+    r = np.zeros((nq, nq))
+    for qb in range(nq):
+        lg = rng.standard_normal(qb + 1) * temp
+        p = np.exp(lg - lg.max())
+        r[qb, : qb + 1] = p / p.sum()
+    return r
+
+
+def test_size_matched_is_heaviest_k_subset_exhaustive():
+    """TopK: the K_q-subset of admissible blocks with the largest step-1 mass (distinct masses:
+    unique), K_q = |W_q| exactly, for random reference rows."""
+    rng = np.random.default_rng(32)
+    nq = 8
+    r1 = _softmax_rows(rng, nq)
+    ref = np.tril(rng.random((nq, nq)) < 0.45)
+    sel = O.size_matched(r1, ref)
+    for qb in range(nq):
+        kq = int(ref[qb].sum())
+        assert sel[qb].sum() == kq and not sel[qb, qb + 1:].any()
+        best = max((sum(r1[qb, list(c)]) for c in itertools.combinations(range(qb + 1), kq)),
+                   default=0.0)
+        assert abs(r1[qb][sel[qb]].sum() - best) < 1e-12
+
+
+def test_size_matched_golden_ties():
+    """Hand-worked: masses (0.25, 0.25, 0.5), K = 2 -> {0, 2} (the tie goes to the lower
+    index); K = 0 -> nothing; K = 3 -> everything."""
+    r1 = np.array([[1.0, 0, 0], [0.5, 0.5, 0], [0.25, 0.25, 0.5]])
+    for k, want in ((2, [0, 2]), (0, []), (3, [0, 1, 2]), (1, [2])):
+        ref = np.zeros((3, 3), bool)
+        ref[2, :k] = True
+        assert np.nonzero(O.size_matched(r1, ref)[2])[0].tolist() == want
+
+
+def test_mass_matched_is_min_cardinality_reaching_wise_mass_exhaustive():
+    """The fewest blocks whose step-1 mass reaches m_q = step-1 mass of W_q; never more blocks
+    than W_q itself (W_q is one such set)."""
+    rng = np.random.default_rng(33)
+    nq = 8
+    r1 = _softmax_rows(rng, nq)
+    ref = np.tril(rng.random((nq, nq)) < 0.5)
+    np.fill_diagonal(ref, True)
+    sel = O.mass_matched(r1, ref)
+    for qb in range(nq):
+        row = r1[qb, : qb + 1]
+        m = math.fsum(row[ref[qb, : qb + 1]])
+        size, best = brute_min_support(row, m)
+        assert sel[qb].sum() == size <= ref[qb].sum()
+        assert abs(row[sel[qb, : qb + 1]].sum() - best) < 1e-12
+        assert math.fsum(row[sel[qb, : qb + 1]]) >= m
+
+
+def test_mass_matched_reproduces_a_ranking_prefix():
+    """If W_q is itself the eta-support of step 1, MassMatched gives back exactly W_q (its
+    mass is reached by the same prefix; no extra block from rounding)."""
+    q, k, _ = rand_qkv(512, 16, 34, scale_q=3.0)
+    r1 = O.block_mass(q, k)
+    for eta in (0.5, 0.9, 0.95, 0.99):
+        w = O.select(r1, eta)
+        assert np.array_equal(O.mass_matched(r1, w), w)
+        assert np.array_equal(O.size_matched(r1, w), w)
+
+
+def test_mass_matched_golden():
+    """Hand-worked: step-1 masses (0.1, 0.2, 0.3, 0.4); W = {0, 1} holds 0.3 of it; the fewest
+    blocks reaching 0.3 are {3} (0.4).  W = {0, 1, 2} holds 0.6 -> {2, 3} (0.7).  Empty W -> {}."""
+    r1 = np.zeros((4, 4))
+    r1[3] = [0.1, 0.2, 0.3, 0.4]
+    r1[:3] = np.tril(np.ones((3, 4))) / np.arange(1, 4)[:, None]
+    for w_row, want in (([0, 1], [3]), ([0, 1, 2], [2, 3]), ([], []), ([3], [3])):
+        ref = np.zeros((4, 4), bool)
+        ref[3, w_row] = True
+        assert np.nonzero(O.mass_matched(r1, ref)[3])[0].tolist() == want
+
+
+def test_static_support_is_a_one_step_window():
+    """Static-95 is the union over the window {1}: the trajectory with window (1, 1)."""
+    cfg = CONFIGS["tiny"]
+    heads = [(0, 0)]
+    steps = [(t, *(bf16_bits_to_f64(x[0]) for x in (q, k, v)))
+             for t, q, k, v in iter_steps(cfg, heads=heads, steps=cfg.t_d)]
+    out = O.head_trajectory(steps, cfg.t_d, (1, 1), 0.95, cfg.scale, keep_dense_o=False)
+    t1, q1, k1, _ = steps[0]
+    assert np.array_equal(out["union"], O.static_support(O.block_mass(q1, k1, cfg.scale)))
+
+
 # --------------------------------------------------------------------------- planted mistakes
 
 def _mutant_attention_no_scale(q, k, v, scale=None, chunk=1024):
@@ -477,3 +600,36 @@ def test_pins_catch_planted_expansion_mistakes():
     want = _element_mask_coarse(sel, factor, n)
     assert np.any(np.triu(_mutant_expand_no_causal_clip(sel, factor), 1))
     assert _element_mask_fine(_mutant_expand_transposed(sel, factor), n) != want
+
+
+def _mutant_size_matched_high_ties(r1, ref):
+    nq = r1.shape[0]
+    sel = np.zeros((nq, nq), dtype=bool)
+    for qb in range(nq):
+        k = int(np.tril(ref)[qb].sum())
+        order = sorted(range(qb + 1), key=lambda b: (-r1[qb, b], -b))
+        sel[qb, order[:k]] = True
+    return sel
+
+
+def _mutant_mass_matched_strict(r1, ref):
+    nq = r1.shape[0]
+    sel = np.zeros((nq, nq), dtype=bool)
+    m = O.retained_mass(r1, ref)
+    for qb in range(nq):
+        row = r1[qb, : qb + 1]
+        order = O.eta_order(row)
+        k = next((k for k in range(qb + 2) if math.fsum(row[order[:k]]) > m[qb]), qb + 1)
+        sel[qb, order[:k]] = True
+    return sel
+
+
+def test_pins_catch_planted_control_mistakes():
+    r1 = np.array([[1.0, 0, 0], [0.5, 0.5, 0], [0.25, 0.25, 0.5]])
+    ref = np.zeros((3, 3), bool)
+    ref[2, :2] = True
+    assert np.nonzero(_mutant_size_matched_high_ties(r1, ref)[2])[0].tolist() != [0, 2]
+    q, k, _ = rand_qkv(512, 16, 34, scale_q=3.0)
+    r = O.block_mass(q, k)
+    w = O.select(r, 0.9)
+    assert not np.array_equal(_mutant_mass_matched_strict(r, w), w)
