@@ -13,6 +13,9 @@
  *                                  wise_select_union_blocks for B = 64 / 128)
  *   once, after step t_d       : wise_build_schedule   (CSR key-block schedule)
  *   late steps t > t_d         : wise_sparse_attn      (block-sparse attention)
+ *   analysis, off the hot path : wise_select_size_matched / _mass_matched
+ *                                  (selection-only controls), wise_support_mass
+ *                                  (retained attention mass of a support)
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -147,6 +150,49 @@ int wise_select_union(const float* mass, uint32_t* union_bits, uint32_t* step_bi
  */
 int wise_select_union_blocks(const float* mass, uint32_t* union_bits, uint32_t* step_bits,
                              float eta, int32_t block, wise_shape_t shape, void* stream);
+
+/*
+ * Selection-only controls (WISE paper appendix B, "Intervention controls").  Both
+ * take the block masses of recurrent step 1 and a reference working set (normally
+ * the WISE union after step t_d) and write a support of the same layout, which
+ * wise_build_schedule turns into a schedule like any other.  (The third control,
+ * Static-95, is wise_select_union on the step-1 masses into a zeroed mask.)
+ *
+ * wise_select_size_matched (SizeMatched): row (bh, q) keeps the K admissible blocks
+ *   of largest mass, K = the number of set admissible bits of the reference row;
+ *   ties go to the lower block index.  K = 0 gives an empty row.
+ * wise_select_mass_matched (MassMatched): m = the fp32 sum of the masses of the
+ *   reference row's set admissible blocks; the row keeps the cumulative-eta support
+ *   at eta = m (rank descending, ties to the lower index, shortest prefix with
+ *   cumulative fp32 mass >= m; m >= 1 keeps every admissible block).  The prefix
+ *   sums use the same summation order as m, so a reference row that is itself a
+ *   ranking prefix is reproduced exactly.  m = 0 gives an empty row.
+ *
+ * mass     : fp32 [B, H, nq, nq] (entries b > q are not read).
+ * ref_bits : uint32 [B, H, nq, W] (bits b > q are ignored).
+ * out_bits : uint32 [B, H, nq, W] output (overwritten, not OR-ed); must not alias
+ *            ref_bits.
+ * Errors   : WISE_ERR_ARG (NULL pointer, aliasing), WISE_ERR_SHAPE, WISE_ERR_CUDA.
+ */
+int wise_select_size_matched(const float* mass, const uint32_t* ref_bits, uint32_t* out_bits,
+                             wise_shape_t shape, void* stream);
+int wise_select_mass_matched(const float* mass, const uint32_t* ref_bits, uint32_t* out_bits,
+                             wise_shape_t shape, void* stream);
+
+/*
+ * Retained attention mass of a support (WISE paper appendix B, "Evaluation
+ * metrics": the fraction of the unrestricted attention mass of a step that falls
+ * inside the frozen support).  retained[bh][q] = sum of mass[bh][q][b] over the
+ * admissible blocks b <= q whose bit is set, in fp32; with the block masses of a
+ * late step and the frozen working set this is the retained future mass of query
+ * block q (the mean over q is the per-token average).
+ *
+ * mass     : fp32 [B, H, nq, nq];  bits : uint32 [B, H, nq, W];
+ * retained : fp32 [B, H, nq] output.
+ * Errors   : WISE_ERR_ARG (NULL pointer), WISE_ERR_SHAPE, WISE_ERR_CUDA.
+ */
+int wise_support_mass(const float* mass, const uint32_t* bits, float* retained,
+                      wise_shape_t shape, void* stream);
 
 /* Workspace bytes wise_build_schedule needs for this shape (device memory). */
 size_t wise_schedule_workspace_bytes(wise_shape_t shape);

@@ -51,6 +51,9 @@ _SIGNATURES = {
     "wise_select_union": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_float, WiseShape, _vp]),
     "wise_select_union_blocks": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_float, ctypes.c_int32,
                                                 WiseShape, _vp]),
+    "wise_select_size_matched": (ctypes.c_int, [_vp, _vp, _vp, WiseShape, _vp]),
+    "wise_select_mass_matched": (ctypes.c_int, [_vp, _vp, _vp, WiseShape, _vp]),
+    "wise_support_mass": (ctypes.c_int, [_vp, _vp, _vp, WiseShape, _vp]),
     "wise_schedule_workspace_bytes": (ctypes.c_size_t, [WiseShape]),
     "wise_schedule_max_nnz": (ctypes.c_int64, [WiseShape]),
     "wise_build_schedule": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int64,

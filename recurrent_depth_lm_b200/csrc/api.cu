@@ -264,6 +264,44 @@ int wise_select_union_blocks(const float* mass, uint32_t* union_bits, uint32_t* 
   return ok();
 }
 
+static int select_control(const float* mass, const uint32_t* ref_bits, uint32_t* out_bits,
+                          int kind, wise_shape_t shape, void* stream, const char* what) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!mass || !ref_bits || !out_bits)
+    return fail(WISE_ERR_ARG, "mass, ref_bits and out_bits must be non-NULL");
+  if (ref_bits == out_bits) return fail(WISE_ERR_ARG, "out_bits must not alias ref_bits");
+  const int nq = shape.seqlen / 32;
+  cudaError_t e = wise::launch_select_control(mass, ref_bits, out_bits, kind,
+                                              shape.batch * shape.heads, nq,
+                                              static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return ok();
+}
+
+int wise_select_size_matched(const float* mass, const uint32_t* ref_bits, uint32_t* out_bits,
+                             wise_shape_t shape, void* stream) {
+  return select_control(mass, ref_bits, out_bits, 0, shape, stream, "select_size_matched launch");
+}
+
+int wise_select_mass_matched(const float* mass, const uint32_t* ref_bits, uint32_t* out_bits,
+                             wise_shape_t shape, void* stream) {
+  return select_control(mass, ref_bits, out_bits, 1, shape, stream, "select_mass_matched launch");
+}
+
+int wise_support_mass(const float* mass, const uint32_t* bits, float* retained,
+                      wise_shape_t shape, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!mass || !bits || !retained)
+    return fail(WISE_ERR_ARG, "mass, bits and retained must be non-NULL");
+  const int nq = shape.seqlen / 32;
+  cudaError_t e = wise::launch_support_mass(mass, bits, retained, shape.batch * shape.heads, nq,
+                                            static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "support_mass launch");
+  return ok();
+}
+
 size_t wise_schedule_workspace_bytes(wise_shape_t shape) {
   if (check_shape(shape)) return 0;
   const long long rows = (long long)shape.batch * shape.heads * (shape.seqlen / 32);

@@ -18,6 +18,7 @@
 // (mass desc, index asc) ranking.
 
 #include <cstdint>
+#include <type_traits>
 
 #include "wise_internal.h"
 
@@ -106,8 +107,8 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Block-size variant (WISE paper appendix C.6, "Block-Size Tradeoff"): selection on blocks of F x 32 tokens,
-// run as exact 32 x 32 subtiles.  One warp per coarse row (bh, Q).  The coarse mass
+// Block-size variant (WISE paper appendix C.6, "Block-Size Tradeoff"): selection on
+// blocks of F x 32 tokens, run as exact 32 x 32 subtiles.  One warp per coarse row (bh, Q).  The coarse mass
 // is the pooled fine mass, R_QB = (1/F) sum_{q in Q} sum_{b in B, b <= q} r_qb, which
 // is the block-mass definition at block size 32F.  After the cut, fine row
 // q = Q F + a keeps fine block b iff coarse block b / F was kept and b <= q.
@@ -234,6 +235,183 @@ cudaError_t launch_select_union_blocks(const float* mass, uint32_t* union_bits,
   if (factor == 2) return launch_pooled<2>(mass, union_bits, step_bits, eta, BH, nq, stream);
   if (factor == 4) return launch_pooled<4>(mass, union_bits, step_bits, eta, BH, nq, stream);
   return cudaErrorInvalidValue;
+}
+
+// ----------------------------------------------------------------------------------------
+// Selection-only controls and the retained-mass metric (WISE paper appendix B,
+// "Intervention controls" and "Evaluation metrics").  One warp per (bh, q) row, the same
+// lane/slot layout as above: lane l holds blocks l, l + 32, ...
+
+template <int MAXW>
+__device__ __forceinline__ void load_mass_row(const float* __restrict__ mrow, int q, int W,
+                                              int lane, float (&v)[MAXW], bool (&ok)[MAXW]) {
+#pragma unroll
+  for (int s = 0; s < MAXW; ++s) {
+    const int kb = s * 32 + lane;
+    ok[s] = (s < W) && (kb <= q);
+    v[s] = ok[s] ? mrow[kb] : 0.f;
+  }
+}
+
+// in[s] = bit (s * 32 + lane) of a [W]-word mask row, admissible blocks only.
+template <int MAXW>
+__device__ __forceinline__ void load_bits_row(const uint32_t* __restrict__ brow,
+                                              const bool (&ok)[MAXW], int lane,
+                                              bool (&in)[MAXW]) {
+#pragma unroll
+  for (int s = 0; s < MAXW; ++s) in[s] = ok[s] && ((brow[s] >> lane) & 1u);
+}
+
+template <int MAXW>
+__device__ __forceinline__ int warp_count_ge(const float (&v)[MAXW], const bool (&ok)[MAXW],
+                                             float tau) {
+  int c = 0;
+#pragma unroll
+  for (int s = 0; s < MAXW; ++s) c += __popc(__ballot_sync(0xffffffffu, ok[s] && v[s] >= tau));
+  return c;
+}
+
+// TopK with ties to the lower index: tau = the largest float with #{v >= tau} >= K, by
+// bisection over the bit patterns (v >= 0); keep v > tau, then blocks equal to tau in
+// ascending index order until K are kept.
+template <int MAXW>
+__device__ __forceinline__ void topk_cut(const float (&v)[MAXW], const bool (&ok)[MAXW], int K,
+                                         int lane, bool (&sel)[MAXW]) {
+  uint32_t lo = 0u, hi = 0x7F800000u;  // count(lo) >= K (every admissible block), count(hi) < K
+  while (hi - lo > 1u) {
+    const uint32_t mid = lo + ((hi - lo) >> 1);
+    if (warp_count_ge<MAXW>(v, ok, __uint_as_float(mid)) >= K)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  const float tau = __uint_as_float(lo);
+  int kept = warp_count_ge<MAXW>(v, ok, __uint_as_float(hi));  // strictly above tau
+#pragma unroll
+  for (int s = 0; s < MAXW; ++s) sel[s] = ok[s] && v[s] > tau;
+#pragma unroll
+  for (int s = 0; s < MAXW; ++s) {
+    uint32_t ties = __ballot_sync(0xffffffffu, ok[s] && v[s] == tau);
+    while (ties != 0u && kept < K) {
+      const int b = __ffs(ties) - 1;
+      ties &= ties - 1u;
+      ++kept;
+      if (lane == b) sel[s] = true;
+    }
+  }
+}
+
+template <int MAXW>
+__device__ __forceinline__ void store_bits_row(uint32_t* __restrict__ dst, int W, int lane,
+                                               const bool (&sel)[MAXW]) {
+  uint32_t word = 0u;
+#pragma unroll
+  for (int s = 0; s < MAXW; ++s) {
+    const uint32_t w = __ballot_sync(0xffffffffu, sel[s]);
+    if (lane == s) word = w;
+  }
+  if (lane < W) dst[lane] = word;
+}
+
+// kSize: SizeMatched, K_q = |W_q| blocks of largest mass.  kMass: MassMatched, the
+// cumulative-eta cut at eta = m_q, the mass of W_q, summed in the same order as the cut's
+// own sums (so a ranking prefix holding W_q's blocks reaches m_q exactly).
+enum ControlKind { kSizeMatched = 0, kMassMatched = 1 };
+
+template <int MAXW, int KIND>
+__global__ void __launch_bounds__(256)
+    select_control_kernel(const float* __restrict__ mass, const uint32_t* __restrict__ ref,
+                          uint32_t* __restrict__ out, long long rows, int nq) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;  // warp-uniform
+  const int W = (nq + 31) >> 5;
+  const int q = (int)(row % nq);
+  float v[MAXW];
+  bool ok[MAXW], in[MAXW], sel[MAXW];
+  load_mass_row<MAXW>(mass + row * (long long)nq, q, W, lane, v, ok);
+  load_bits_row<MAXW>(ref + row * W, ok, lane, in);
+  if (KIND == kSizeMatched) {
+    int K = 0;
+#pragma unroll
+    for (int s = 0; s < MAXW; ++s) K += __popc(__ballot_sync(0xffffffffu, in[s]));
+    if (K == 0) {
+#pragma unroll
+      for (int s = 0; s < MAXW; ++s) sel[s] = false;
+    } else {
+      topk_cut<MAXW>(v, ok, K, lane, sel);
+    }
+  } else {
+    const float m = warp_sum_ge<MAXW>(v, in, 0.f);
+    if (!(m > 0.f)) {
+#pragma unroll
+      for (int s = 0; s < MAXW; ++s) sel[s] = false;
+    } else {
+      eta_cut<MAXW>(v, ok, m, lane, sel);
+    }
+  }
+  store_bits_row<MAXW>(out + row * W, W, lane, sel);
+}
+
+// retained[row] = sum of mass[row][b] over set bits b <= q (fp32, same order as above).
+template <int MAXW>
+__global__ void __launch_bounds__(256)
+    support_mass_kernel(const float* __restrict__ mass, const uint32_t* __restrict__ bits,
+                        float* __restrict__ retained, long long rows, int nq) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;  // warp-uniform
+  const int W = (nq + 31) >> 5;
+  const int q = (int)(row % nq);
+  float v[MAXW];
+  bool ok[MAXW], in[MAXW];
+  load_mass_row<MAXW>(mass + row * (long long)nq, q, W, lane, v, ok);
+  load_bits_row<MAXW>(bits + row * W, ok, lane, in);
+  const float m = warp_sum_ge<MAXW>(v, in, 0.f);
+  if (lane == 0) retained[row] = m;
+}
+
+// Calls f(std::integral_constant<int, MAXW>) for the smallest MAXW in {1, 2, 4, 8, 16} >= W.
+template <typename Fn>
+static cudaError_t by_width(int W, Fn&& f) {
+  if (W <= 1)
+    f(std::integral_constant<int, 1>{});
+  else if (W <= 2)
+    f(std::integral_constant<int, 2>{});
+  else if (W <= 4)
+    f(std::integral_constant<int, 4>{});
+  else if (W <= 8)
+    f(std::integral_constant<int, 8>{});
+  else if (W <= 16)
+    f(std::integral_constant<int, 16>{});
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_control(const float* mass, const uint32_t* ref_bits, uint32_t* out_bits,
+                                  int kind, int BH, int nq, cudaStream_t stream) {
+  const long long rows = (long long)BH * nq;
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  return by_width((nq + 31) / 32, [&](auto w) {
+    constexpr int M = decltype(w)::value;
+    if (kind == kSizeMatched)
+      select_control_kernel<M, kSizeMatched><<<grid, 256, 0, stream>>>(mass, ref_bits, out_bits,
+                                                                       rows, nq);
+    else
+      select_control_kernel<M, kMassMatched><<<grid, 256, 0, stream>>>(mass, ref_bits, out_bits,
+                                                                       rows, nq);
+  });
+}
+
+cudaError_t launch_support_mass(const float* mass, const uint32_t* bits, float* retained, int BH,
+                                int nq, cudaStream_t stream) {
+  const long long rows = (long long)BH * nq;
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  return by_width((nq + 31) / 32, [&](auto w) {
+    constexpr int M = decltype(w)::value;
+    support_mass_kernel<M><<<grid, 256, 0, stream>>>(mass, bits, retained, rows, nq);
+  });
 }
 
 }  // namespace wise

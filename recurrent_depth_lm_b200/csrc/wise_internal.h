@@ -48,6 +48,15 @@ cudaError_t launch_select_union_blocks(const float* mass, uint32_t* union_bits,
                                        uint32_t* step_bits, float eta, int factor, int BH, int nq,
                                        cudaStream_t stream);
 
+// Selection-only controls from a reference mask: kind 0 = SizeMatched (TopK, K = |ref row|),
+// kind 1 = MassMatched (cumulative cut at the mass of the ref row).
+cudaError_t launch_select_control(const float* mass, const uint32_t* ref_bits, uint32_t* out_bits,
+                                  int kind, int BH, int nq, cudaStream_t stream);
+
+// retained[bh * nq + q] = sum of mass over the set admissible bits of the row.
+cudaError_t launch_support_mass(const float* mass, const uint32_t* bits, float* retained, int BH,
+                                int nq, cudaStream_t stream);
+
 size_t schedule_workspace_bytes(long long rows);
 cudaError_t launch_build_schedule(const uint32_t* union_bits, int32_t* row_offsets,
                                   int32_t* col_idx, long long capacity, void* workspace,

@@ -106,6 +106,40 @@ def select_union(mass, union_bits, eta: float, *, step_bits=None, head_dim: int 
     return union_bits
 
 
+def _control(fn, name, mass, ref_bits, out, head_dim, stream):
+    b, h, nq, _ = mass.shape
+    if mass.dtype != torch.float32 or ref_bits.dtype != torch.int32:
+        raise ValueError("mass must be float32 and ref_bits int32 (uint32 bit patterns)")
+    out = torch.empty_like(ref_bits) if out is None else out
+    shp = WiseShape(b, h, nq * BLOCK, head_dim, 0.0)
+    check(fn(_ptr(mass), _ptr(ref_bits), _ptr(out), shp, _stream(stream)), name)
+    return out
+
+
+def select_size_matched(mass, ref_bits, *, out=None, head_dim: int = 128, stream=None):
+    """SizeMatched control: per row the |ref row| blocks of largest mass (TopK)."""
+    return _control(lib.wise_select_size_matched, "wise_select_size_matched", mass, ref_bits,
+                    out, head_dim, stream)
+
+
+def select_mass_matched(mass, ref_bits, *, out=None, head_dim: int = 128, stream=None):
+    """MassMatched control: per row the fewest ranked blocks reaching the ref row's mass."""
+    return _control(lib.wise_select_mass_matched, "wise_select_mass_matched", mass, ref_bits,
+                    out, head_dim, stream)
+
+
+def support_mass(mass, bits, *, out=None, head_dim: int = 128, stream=None):
+    """Retained attention mass of the support `bits` per (b, h, q): fp32 [B, H, nq]."""
+    b, h, nq, _ = mass.shape
+    if mass.dtype != torch.float32 or bits.dtype != torch.int32:
+        raise ValueError("mass must be float32 and bits int32 (uint32 bit patterns)")
+    out = torch.empty(b, h, nq, dtype=torch.float32, device=mass.device) if out is None else out
+    shp = WiseShape(b, h, nq * BLOCK, head_dim, 0.0)
+    check(lib.wise_support_mass(_ptr(mass), _ptr(bits), _ptr(out), shp, _stream(stream)),
+          "wise_support_mass")
+    return out
+
+
 def new_bitmask(b: int, h: int, nq: int, device) -> torch.Tensor:
     return torch.zeros(b, h, nq, words_per_row(nq), dtype=torch.int32, device=device)
 

@@ -9,6 +9,14 @@ step runs block-sparse attention over that schedule with fresh Q, K, V.
 Appendix C.6's block-size variants (block = 64 or 128) select on coarser blocks
 and run the result as exact 32 x 32 subtiles.
 
+The selection-only controls of appendix B ("Intervention controls") replace the
+frozen support: "static95" is the eta-support of step 1 alone, "size_matched"
+the |W_q| blocks of largest step-1 mass, "mass_matched" the fewest step-1-ranked
+blocks reaching the step-1 mass of W_q; steps up to t_d are unchanged.  With
+track_retained, every late step also runs dense attention with block mass
+(analysis only) and records the retained future mass of the frozen support
+("Evaluation metrics").
+
 All buffers are allocated once here with torch; the library calls only
 enqueue kernels on the current stream (no host synchronisation inside a
 trajectory).
@@ -20,11 +28,18 @@ import torch
 
 from . import ops
 
+SUPPORTS = ("wise", "static95", "size_matched", "mass_matched")
+
 
 class WiseTrajectory:
     def __init__(self, batch: int, heads: int, seqlen: int, head_dim: int, *, t_d: int = 12,
                  window=(9, 12), eta: float = 0.95, scale: float | None = None,
-                 block: int = ops.BLOCK, device="cuda", keep_step_bits: bool = False):
+                 block: int = ops.BLOCK, support: str = "wise", track_retained: bool = False,
+                 device="cuda", keep_step_bits: bool = False):
+        if support not in SUPPORTS:
+            raise ValueError(f"support must be one of {SUPPORTS}")
+        if support in ("size_matched", "mass_matched") and block != ops.BLOCK:
+            raise ValueError("the size- and mass-matched controls are defined for block = 32")
         if block not in (32, 64, 128):
             raise ValueError("block must be 32, 64 or 128")
         if seqlen % block:
@@ -47,11 +62,29 @@ class WiseTrajectory:
                                    dtype=torch.int32, device=dev)
         self.workspace = ops.schedule_workspace(batch, heads, seqlen, head_dim, dev)
         self.scheduled = False
+        self.support = support
+        # step-1 block masses and the control support (selection-only controls)
+        self.mass1 = (torch.empty_like(self.mass) if support != "wise" else None)
+        self.control = ops.new_bitmask(batch, heads, self.nq, dev) if support != "wise" else None
+        self.track_retained = track_retained
+        self.retained = {}
+        self.o_scratch = None
+        if track_retained:
+            self.o_scratch = torch.empty(batch, heads, seqlen, head_dim, dtype=torch.bfloat16,
+                                         device=dev)
 
     def reset(self) -> None:
         self.union.zero_()
+        if self.control is not None:
+            self.control.zero_()
         self.step_bits.clear()
+        self.retained.clear()
         self.scheduled = False
+
+    @property
+    def frozen(self):
+        """The support the late steps run on (the WISE union or the control)."""
+        return self.union if self.support == "wise" else self.control
 
     def in_window(self, t: int) -> bool:
         return self.window[0] <= t <= self.window[1]
@@ -59,17 +92,22 @@ class WiseTrajectory:
     def step(self, t: int, q, k, v, o=None, lse=None, stream=None):
         """Attention of recurrent step t (1-based).  Returns O."""
         if t <= self.t_d:
-            if self.in_window(t):
-                o, _, _ = ops.full_attn_mass(q, k, v, o=o, lse=self.lse, mass=self.mass,
+            first = t == 1 and self.mass1 is not None   # step-1 masses for the controls
+            if self.in_window(t) or first:
+                m = self.mass1 if first else self.mass
+                o, _, _ = ops.full_attn_mass(q, k, v, o=o, lse=self.lse, mass=m,
                                              workspace=self.mass_ws, scale=self.scale,
                                              stream=stream)
-                sb = None
-                if self.keep_step_bits:
-                    sb = torch.empty_like(self.union)
-                    self.step_bits[t] = sb
-                ops.select_union(self.mass, self.union, self.eta, step_bits=sb,
-                                 head_dim=self.d, scale=self.scale, block=self.block,
-                                 stream=stream)
+                if self.in_window(t):
+                    sb = None
+                    if self.keep_step_bits:
+                        sb = torch.empty_like(self.union)
+                        self.step_bits[t] = sb
+                    ops.select_union(m, self.union, self.eta, step_bits=sb, head_dim=self.d,
+                                     scale=self.scale, block=self.block, stream=stream)
+                if first and self.support == "static95":
+                    ops.select_union(m, self.control, self.eta, head_dim=self.d,
+                                     scale=self.scale, block=self.block, stream=stream)
             else:
                 o, _, _ = ops.full_attn_mass(q, k, v, o=o, lse=lse, scale=self.scale,
                                              stream=stream)
@@ -80,13 +118,30 @@ class WiseTrajectory:
             raise RuntimeError("late step before the schedule was built (t <= t_d never reached)")
         o, _ = ops.sparse_attn(q, k, v, self.row_offsets, self.col_idx, self.col_idx.numel(),
                                o=o, lse=lse, scale=self.scale, stream=stream)
+        if self.track_retained:
+            ops.full_attn_mass(q, k, v, o=self.o_scratch, lse=self.lse, mass=self.mass,
+                               workspace=self.mass_ws, scale=self.scale, stream=stream)
+            self.retained[t] = ops.support_mass(self.mass, self.frozen, head_dim=self.d,
+                                                stream=stream)
         return o
 
     def build_schedule(self, stream=None) -> None:
-        ops.build_schedule(self.union, head_dim=self.d, row_offsets=self.row_offsets,
+        if self.support == "size_matched":
+            ops.select_size_matched(self.mass1, self.union, out=self.control, head_dim=self.d,
+                                    stream=stream)
+        elif self.support == "mass_matched":
+            ops.select_mass_matched(self.mass1, self.union, out=self.control, head_dim=self.d,
+                                    stream=stream)
+        ops.build_schedule(self.frozen, head_dim=self.d, row_offsets=self.row_offsets,
                            col_idx=self.col_idx, workspace=self.workspace, exact_nnz=False,
                            stream=stream)
         self.scheduled = True
+
+    def retained_future_mass(self) -> float:
+        """Mean over late steps, heads and query blocks of the retained attention mass."""
+        if not self.retained:
+            raise RuntimeError("no late step ran with track_retained=True")
+        return float(torch.stack(list(self.retained.values())).mean().item())
 
     def nnz(self) -> int:
         return int(self.row_offsets[-1].item())

@@ -115,6 +115,23 @@ def test_select_blocks_checks(lib):
     assert L.wise_select_union_blocks(fake, fake, None, 0.95, 128, odd, None) == \
         lib.WISE_ERR_SHAPE
 
+
+def test_control_and_support_mass_checks(lib):
+    L = lib.lib
+    s = shape(lib)
+    a, b = 1 << 20, 1 << 21
+    for fn in (L.wise_select_size_matched, L.wise_select_mass_matched):
+        assert fn(None, a, b, s, None) == lib.WISE_ERR_ARG
+        assert fn(a, None, b, s, None) == lib.WISE_ERR_ARG
+        assert fn(a, b, None, s, None) == lib.WISE_ERR_ARG
+        assert fn(a, b, b, s, None) == lib.WISE_ERR_ARG          # out aliases ref
+        assert "alias" in lib.last_error()
+        assert fn(a, b, a + 64, lib.WiseShape(1, 2, 100, 64, 0.0, 0), None) == lib.WISE_ERR_SHAPE
+    assert L.wise_support_mass(None, a, b, s, None) == lib.WISE_ERR_ARG
+    assert L.wise_support_mass(a, b, None, s, None) == lib.WISE_ERR_ARG
+    assert L.wise_support_mass(a, b, a + 64, lib.WiseShape(1, 2, 256, 80, 0.0, 0), None) == \
+        lib.WISE_ERR_SHAPE
+
 def test_schedule_sizes_and_checks(lib):
     L = lib.lib
     s = shape(lib, 1, 32, 4096, 128)

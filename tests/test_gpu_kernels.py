@@ -435,6 +435,92 @@ def test_select_union_blocks_32_is_the_plain_selection(ops):
     torch.cuda.synchronize()
     assert torch.equal(a, b)
 
+
+# ---------------------------------------------------------------- controls and retained mass
+
+def _bits_of(sel):
+    """[bh, nq, nq] bool -> [1, bh, nq, W] int32 device words."""
+    bh, nq, _ = sel.shape
+    W = (nq + 31) // 32
+    words = np.zeros((bh, nq, W), np.uint32)
+    for b in range(nq):
+        words[..., b // 32] |= sel[..., b].astype(np.uint32) << np.uint32(b % 32)
+    return torch.from_numpy(words.view(np.int32)).reshape(1, bh, nq, W).cuda()
+
+
+def _control_inputs(nq, bh, seed):
+    rng = np.random.default_rng(seed)
+    m32 = _peaky_masses(rng, bh, nq).astype(np.float32)
+    ref = rng.random((bh, nq, nq)) < 0.3
+    ref[:, np.arange(nq), np.arange(nq)] = True
+    ref[0, nq // 2] = False                 # one empty reference row
+    ref |= np.triu(np.ones((nq, nq), bool), 1)   # bits b > q are set and must be ignored
+    return m32, ref
+
+
+@pytest.mark.parametrize("nq,bh", [(8, 2), (45, 3), (128, 2), (512, 1)])
+def test_size_matched_bit_exact(ops, nq, bh):
+    """TopK involves only comparisons of the same fp32 masses: bit-exact against the oracle."""
+    m32, ref = _control_inputs(nq, bh, 40 + nq)
+    out = ops.select_size_matched(torch.from_numpy(m32).reshape(1, bh, nq, nq).cuda(), _bits_of(ref))
+    got = bits_to_bool(out.cpu().numpy()[0], nq)
+    for x in range(bh):
+        want = O.size_matched(m32[x].astype(np.float64), ref[x])
+        assert np.array_equal(got[x], want)
+        assert np.array_equal(got[x].sum(axis=1), np.tril(ref[x]).sum(axis=1))
+
+
+def test_size_matched_ties_go_to_lower_index(ops):
+    nq = 40
+    m = np.tril(np.full((nq, nq), 1.0, np.float32))
+    m /= m.sum(axis=1, keepdims=True)       # uniform rows: every admissible block ties
+    ref = np.zeros((1, nq, nq), bool)
+    for qb in range(nq):
+        ref[0, qb, : (qb + 1) // 2 + 1] = True
+    out = ops.select_size_matched(torch.from_numpy(m).reshape(1, 1, nq, nq).cuda(), _bits_of(ref))
+    got = bits_to_bool(out.cpu().numpy()[0], nq)[0]
+    for qb in range(nq):
+        k = (qb + 1) // 2 + 1
+        assert np.nonzero(got[qb])[0].tolist() == list(range(min(k, qb + 1)))
+
+
+@pytest.mark.parametrize("nq,bh", [(8, 2), (45, 3), (128, 2), (512, 1)])
+def test_mass_matched_matches_oracle(ops, nq, bh):
+    m32, ref = _control_inputs(nq, bh, 50 + nq)
+    dm = torch.from_numpy(m32).reshape(1, bh, nq, nq).cuda()
+    got = bits_to_bool(ops.select_mass_matched(dm, _bits_of(ref)).cpu().numpy()[0], nq)
+    exempt = 0
+    for x in range(bh):
+        r = m32[x].astype(np.float64)
+        want = O.mass_matched(r, ref[x])
+        for qb in range(nq):
+            if np.array_equal(got[x, qb], want[qb]):
+                continue
+            row = r[qb, : qb + 1]
+            m = O.retained_mass(r, ref[x])[qb]
+            d_ck, d_ck1, r_cut = O.cut_margins(row, m)
+            assert not got[x, qb, qb + 1:].any()
+            assert min(d_ck, d_ck1) <= 1e-5, (x, qb)   # fp32 sums vs correctly rounded ones
+            exempt += 1
+        # a reference that is itself a ranking prefix comes back exactly
+        w = O.select(r, 0.9)
+        back = ops.select_mass_matched(dm[:, x:x + 1].contiguous(), _bits_of(w[None]))
+        assert np.array_equal(bits_to_bool(back.cpu().numpy()[0], nq)[0], w)
+    assert exempt <= 2
+
+
+@pytest.mark.parametrize("nq,bh", [(8, 2), (45, 3), (512, 1)])
+def test_support_mass_matches_oracle(ops, nq, bh):
+    """fp32 sum of <= 512 non-negative masses with total <= 1: error <= 21 * 2^-24 (16
+    sequential adds per lane, a 5-level tree), 2e-6 with margin."""
+    m32, ref = _control_inputs(nq, bh, 60 + nq)
+    out = ops.support_mass(torch.from_numpy(m32).reshape(1, bh, nq, nq).cuda(), _bits_of(ref))
+    got = out.cpu().numpy()[0]
+    for x in range(bh):
+        want = O.retained_mass(m32[x].astype(np.float64), ref[x])
+        assert np.abs(got[x] - want).max() <= 2e-6
+    assert got[0, nq // 2] == 0.0
+
 @pytest.mark.parametrize("nq,bh", [(1, 1), (8, 2), (45, 3), (512, 2)])
 def test_build_schedule_bit_exact(ops, nq, bh):
     rng = np.random.default_rng(nq * 7 + bh)

@@ -140,3 +140,85 @@ def test_trajectory_2k_b4_h40_d96():
 def test_trajectory_16k_and_eta_one():
     cfg = CONFIGS["16k"]
     check_config(cfg, [(0, 5)], check_steps=[12, 13, 32], etas=(None, 1.0))
+
+
+# ------------------------------------------------------------- selection-only controls
+
+def _size_matched_near_tie(row, k):
+    """The K-th and (K+1)-th largest masses are within the mass tolerance (TopK may flip)."""
+    srt = np.sort(row)[::-1]
+    return 0 < k < len(srt) and srt[k - 1] - srt[k] <= MASS_TOL
+
+
+@pytest.mark.parametrize("support", ["wise", "static95", "size_matched", "mass_matched"])
+def test_trajectory_controls_and_retained_mass(support):
+    """Late steps on a control support (appendix B "Intervention controls") with the retained
+    future mass tracked.  The control is checked against the oracle's control computed from
+    the oracle's step-1 masses and the GPU's own union (so a near-cut flip in the union does
+    not cascade); the schedule, late O and per-row retained mass against the oracle."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from recurrent_depth_lm_b200 import WiseTrajectory, ops
+    cfg = CONFIGS["1k"]
+    sample = [(0, 0), (0, 31)]
+    idx = [b * cfg.heads + h for (b, h) in sample]
+    nq = cfg.nq
+    check_steps = [13, 20, 32]
+    tr = WiseTrajectory(cfg.batch, cfg.heads, cfg.seqlen, cfg.head_dim, t_d=cfg.t_d,
+                        window=cfg.window, eta=cfg.eta, support=support, track_retained=True)
+    flat = lambda x: x.reshape(cfg.bh, *x.shape[2:])[idx]
+    o_late, retained = {}, {}
+    with StepPool(cfg, workers=max(1, min(16, os.cpu_count() or 2))) as pool:
+        for t, q, k, v in pool:
+            o = tr.step(t, _dev(q), _dev(k), _dev(v))
+            if t == 1 and tr.mass1 is not None:
+                mass1 = flat(tr.mass1).cpu().numpy()
+            if t in check_steps:
+                o_late[t] = flat(o).float().cpu().numpy()
+            if t > cfg.t_d:
+                retained[t] = flat(tr.retained[t]).cpu().numpy()
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    union = bits_to_bool(flat(tr.union).cpu().numpy(), nq)
+    frozen = bits_to_bool(flat(tr.frozen).cpu().numpy(), nq)
+    ro_all, ci_all = tr.row_offsets.cpu().numpy(), tr.col_idx.cpu().numpy()
+    host = {t: (q, k, v) for t, q, k, v in iter_steps(cfg, heads=sample)}
+    exempt = 0
+    for si, bhi in enumerate(idx):
+        ro = ro_all[bhi * nq:(bhi + 1) * nq + 1] - ro_all[bhi * nq]
+        ci = ci_all[ro_all[bhi * nq]:ro_all[(bhi + 1) * nq]]
+        check_csr(ro, ci, frozen[si])
+        if support != "wise":
+            q1, k1, _ = (bf16_bits_to_f64(x[si]) for x in host[1])
+            r1 = O.block_mass(q1, k1, cfg.scale)
+            assert np.abs(np.tril(mass1[si]) - r1).max() <= MASS_TOL
+            if support == "static95":
+                exempt += compare_selection(frozen[si], r1, cfg.eta)
+            else:
+                want = (O.size_matched if support == "size_matched" else O.mass_matched)(
+                    r1, union[si])
+                for qb in range(nq):
+                    if np.array_equal(frozen[si, qb], want[qb]):
+                        continue
+                    row = r1[qb, : qb + 1]
+                    if support == "size_matched":
+                        assert frozen[si, qb].sum() == np.tril(union[si])[qb].sum()
+                        assert _size_matched_near_tie(row, int(want[qb].sum())), qb
+                    else:
+                        m = O.retained_mass(r1, union[si])[qb]
+                        d_ck, d_ck1, _ = O.cut_margins(row, m)
+                        assert min(d_ck, d_ck1) <= 1e-4, qb
+                    exempt += 1
+        else:
+            assert np.array_equal(frozen[si], union[si])
+        for t in range(cfg.t_d + 1, cfg.steps + 1):
+            if t not in check_steps:
+                continue
+            q, k, v = (bf16_bits_to_f64(x[si]) for x in host[t])
+            ref, _ = O.masked_attention(q, k, v, frozen[si], cfg.scale)
+            compare_o(o_late[t][si], ref, f"{support} head {sample[si]} step {t}")
+            want_ret = O.retained_mass(O.block_mass(q, k, cfg.scale), frozen[si])
+            assert np.abs(retained[t][si] - want_ret).max() <= MASS_TOL
+    assert exempt <= 3
+    rfm = tr.retained_future_mass()
+    assert 0.0 < rfm <= 1.0 + 1e-6
