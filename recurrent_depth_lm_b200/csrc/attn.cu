@@ -67,7 +67,8 @@ struct Entry {
   int bh;
   int Qt;
   int stage;   // index among the CTA's work entries: K ring = stage % NK, V ring = stage % NV
-  int pad0, pad1;
+  int kvh;     // K/V head of bh (bh / group), computed once per tile
+  int pad0;
   int kb[kSlots];
   int own[kSlots];
 };
@@ -365,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     struct Slot {
       DenseList dl;
       MaskList ml;
-      int bh, qt, rc;
+      int bh, qt, rc, kvh;
       uint32_t tq;          // tiles started (q_empty phases)
       bool active, ended, first;
     };
@@ -391,6 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         }
         decode_tile(tile, p.BH, ntq, S.bh, S.qt);
+        S.kvh = S.bh / p.group;
         if (MODE == kModeSparse) {
           uint32_t* msk = masks + X * 4 * kMaxWords;
           build_tile_masks(msk, p, S.bh, S.qt, lane);
@@ -436,6 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         e.flags = (S.first ? kFirst : 0) | (last ? kLast : 0);
         e.ns = n;
         e.bh = S.bh;
+        e.kvh = S.kvh;
         e.Qt = S.qt;
         e.stage = (int)g;
         for (int s = 0; s < kSlots; ++s) {
@@ -451,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int pn = 0; pn < C::kPanels; ++pn)
             tma_load_3d(kbase + pn * kPanelBytes + s * 32 * kPanelRowBytes, &tmK, bar_k_full(ks),
-                        pn * 64, kb * 32, S.bh / p.group);
+                        pn * 64, kb * 32, S.kvh);
         }
       }
       ++S.rc;
@@ -494,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Entry& e = ents[X * kRing + k];
         const int kind = e.kind;
         const int n = e.ns;
-        const int bh = e.bh;
+        const int kvh = e.kvh;
         const uint32_t g = (uint32_t)e.stage;
         int kbv[kSlots];
 #pragma unroll
@@ -517,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int pn = 0; pn < C::kPanels; ++pn)
             tma_load_3d(vbase + pn * kPanelBytes + s * 32 * kPanelRowBytes, &tmV, bar_v_full(vs),
-                        pn * 64, kb * 32, bh / p.group);
+                        pn * 64, kb * 32, kvh);
         }
         issued = g + 1;
         return true;
