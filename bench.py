@@ -325,6 +325,25 @@ def run_e2e(cfg, runner, host_q, host_k, host_v, reps: int):
     return dt, 3 * T * per, T * per
 
 
+def routing_stats(cfg, q, k, v, device, block: int = 32):
+    """Untimed: block density and retained future attention mass (WISE paper appendix B,
+    "Evaluation metrics") of the WISE working set and of the selection-only controls,
+    each from one trajectory over the same inputs with the late-step mass tracked."""
+    from recurrent_depth_lm_b200.trajectory import WiseTrajectory
+    out = {}
+    supports = ["wise", "static95"] + (["size_matched", "mass_matched"] if block == 32 else [])
+    for support in supports:
+        tr = WiseTrajectory(cfg.batch, cfg.heads, cfg.seqlen, cfg.head_dim, t_d=cfg.t_d,
+                            window=cfg.window, eta=cfg.eta, block=block, support=support,
+                            track_retained=True, device=device)
+        for t in range(1, cfg.steps + 1):
+            tr.step(t, q[t - 1], k[t - 1], v[t - 1])
+        out[support] = {"density": round(tr.density(), 4),
+                        "retained_future_mass": round(tr.retained_future_mass(), 4)}
+        del tr
+    return out
+
+
 def cpu_oracle_sample(cfg, n_heads: int = 1, block: int = 32):
     """The CPU oracle, as it stands, on a bounded sample: for each sampled head one
     exploration step (dense attention + block mass + eta-selection -> schedule) and
@@ -367,16 +386,33 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
+def workload(args):
+    """The named workload with the one-at-a-time overrides (eta, t_d, window) applied."""
+    from wise_inputs import CONFIGS
+    cfg = CONFIGS[args.config]
+    kw = {}
+    if args.eta is not None:
+        kw["eta"] = args.eta
+    if args.t_d is not None:
+        kw["t_d"] = args.t_d
+        kw["window"] = (max(1, args.t_d - 3), args.t_d)
+    if args.window is not None:
+        kw["window"] = tuple(args.window)
+    cfg = cfg.with_(**kw) if kw else cfg
+    if not (1 <= cfg.window[0] <= cfg.window[1] <= cfg.t_d < cfg.steps):
+        raise SystemExit(f"bad discovery window {cfg.window} for t_d={cfg.t_d}, T={cfg.steps}")
+    return cfg
+
+
 def bench_wise(args):
     import numpy as np
     import torch
-    from wise_inputs import CONFIGS
 
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     init_dist(world, "nccl")
-    cfg = CONFIGS[args.config]
+    cfg = workload(args)
     workers = args.workers or max(1, min(16, (os.cpu_count() or 2) // max(1, world)))
 
     q, k, v, _ = make_inputs(cfg, rank, device, workers)
@@ -442,6 +478,8 @@ def bench_wise(args):
                 "traffic": profiled_traffic(kname, cfg.name),
                 "flops_per_launch": k_flops}
 
+    routing = routing_stats(cfg, q, k, v, device, args.block) if args.routing else None
+
     e2e = None
     if args.e2e:
         shp = (cfg.steps, cfg.batch, cfg.heads, cfg.seqlen, cfg.head_dim)
@@ -486,6 +524,7 @@ def bench_wise(args):
         "select_us": round(sel_us, 2) if sel_us else None,
         "schedule_us": round(sched_us, 2) if sched_us else None,
         "density": round(density, 4), "nnz_blocks": nnz,
+        "routing": routing,
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
         "gpu_launches": runner.launches_per_trajectory() * args.steps,
         "device_status": status,
@@ -503,8 +542,7 @@ def bench_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
         return
-    from wise_inputs import CONFIGS
-    cfg = CONFIGS[args.config]
+    cfg = workload(args)
     for _ in range(args.warmup):
         cpu_oracle_sample(cfg, n_heads=1, block=args.block)
     secs, flops = 0.0, 0.0
@@ -520,7 +558,8 @@ def bench_reference(args):
         "ms_per_step": round(secs / args.steps * 1e3, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "impl": "reference",
         "data": "synthetic (seeded generator)",
-        "config": {"workload": f"{cfg.name}, B={args.block}",
+        "config": {"workload": f"{cfg.name}, dense 1-{cfg.t_d}, union {cfg.window[0]}-"
+                               f"{cfg.window[1]}, eta={cfg.eta}, B={args.block}",
                    "step": "bounded oracle sample (see cpu_baseline)"},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "kind": "oracle",
                          "cores": blas_threads(), "sample": desc},
@@ -539,12 +578,20 @@ def main(argv=None):
     ap.add_argument("--config", default="4k")
     ap.add_argument("--block", type=int, choices=[32, 64, 128], default=32,
                     help="selection block size (64 / 128 run as 32x32 subtiles)")
+    ap.add_argument("--eta", type=float, default=None,
+                    help="mass threshold (default: the workload's, 0.95)")
+    ap.add_argument("--t-d", dest="t_d", type=int, default=None,
+                    help="discovery depth: last dense step (default 12)")
+    ap.add_argument("--window", type=int, nargs=2, default=None, metavar=("FIRST", "LAST"),
+                    help="discovery window (default: the last four steps up to t_d)")
     ap.add_argument("--workers", type=int, default=0)
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--e2e-reps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-heads", type=int, default=16)
     ap.add_argument("--no-clocks", dest="clocks", action="store_false")
+    ap.add_argument("--no-routing", dest="routing", action="store_false",
+                    help="skip the untimed density / retained-future-mass pass")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

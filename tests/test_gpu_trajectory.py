@@ -127,6 +127,23 @@ def test_trajectory_1k_block_sizes(block):
     assert rep[None]["exempt_rows"] <= 2
 
 
+# One-at-a-time variants of the frozen configuration (WISE paper appendix C.5, Table 7,
+# and C.7, Table 9): the mass threshold, the discovery depth and the union width.
+VARIANTS = [
+    dict(eta=0.90), dict(eta=0.98), dict(eta=0.99),
+    dict(t_d=8, window=(5, 8)), dict(t_d=16, window=(13, 16)),
+    dict(window=(12, 12)), dict(window=(11, 12)),
+]
+
+
+@pytest.mark.parametrize("variant", VARIANTS, ids=lambda v: "-".join(f"{k}{v[k]}" for k in v))
+def test_trajectory_1k_hyperparameter_variants(variant):
+    cfg = CONFIGS["1k"].with_(**variant)
+    late = [cfg.t_d + 1, cfg.steps]
+    rep = check_config(cfg, [(0, 3), (0, 30)], check_steps=late)
+    assert rep[None]["exempt_rows"] <= 2
+
+
 def test_trajectory_4k():
     cfg = CONFIGS["4k"]
     check_config(cfg, [(0, 0), (0, 21)], check_steps=[1, 9, 12, 13, 20, 32])
