@@ -201,28 +201,34 @@ def support_from_csr(row_offsets, col_idx, nq: int) -> np.ndarray:
     return sup
 
 
-def masked_attention(q, k, v, support: np.ndarray, scale=None, chunk: int = 1024):
+def masked_attention(q, k, v, support: np.ndarray, scale=None, chunk: int = 1024,
+                     block: int = BLOCK):
     """Attention under the reuse mask R of WISE paper §5.2 plus the causal mask M.
 
-    R_ij = 0 if b(j) is in the support of q(i), else -inf.  Returns (O, lse).
-    Skipping absent blocks (§7.4, App. B) is exactly this masked softmax.
+    R_ij = 0 if b(j) is in the support of q(i), else -inf, with blocks of ``block``
+    tokens (32, or another size of App. C.6; ``support`` is [n/block, n/block]).
+    Returns (O, lse).  Skipping absent blocks (§7.4, App. B) is exactly this masked
+    softmax.  A row with no admissible kept key has O = 0 and lse = -inf.
     """
     q, k, v = (np.asarray(x, np.float64) for x in (q, k, v))
     n = q.shape[0]
     scale = default_scale(q.shape[1]) if scale is None else float(scale)
     o = np.empty_like(q)
     lse = np.empty(n)
-    blk = np.arange(n) // BLOCK
+    blk = np.arange(n) // block
     for r0 in range(0, n, chunk):
         rows = slice(r0, min(n, r0 + chunk))
         s = _causal_scores(q, k, scale, rows)
         allowed = support[blk[rows]][:, blk]          # [rows, n]: b(j) in B_q(i)
         s[~allowed] = -np.inf
         m = s.max(axis=1, keepdims=True)
+        empty = ~np.isfinite(m[:, 0])                 # no kept admissible key in the row
+        m[empty] = 0.0
         p = np.exp(s - m)
         l = p.sum(axis=1, keepdims=True)
+        l[empty] = 1.0
         o[rows] = (p / l) @ v
-        lse[rows] = (m + np.log(l))[:, 0]
+        lse[rows] = np.where(empty, -np.inf, (m + np.log(l))[:, 0])
     return o, lse
 
 

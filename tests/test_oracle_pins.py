@@ -171,9 +171,9 @@ def test_block_mass_equals_blocks_of_attention_matrix():
 
 # --------------------------------------------------------------------------- block-size variants
 
-@pytest.mark.parametrize("block", [64, 128])
+@pytest.mark.parametrize("block", [16, 64, 128])
 def test_block_mass_uniform_closed_form_larger_blocks(block):
-    """Q = 0 at B = 64 / 128: r_QB = mean_i |I_B cap [0, i]| / (i + 1), exact fractions."""
+    """Q = 0 at B = 16 / 64 / 128: r_QB = mean_i |I_B cap [0, i]| / (i + 1), exact fractions."""
     nb = 3
     n = nb * block
     _, k, _ = rand_qkv(n, 4, 18)
@@ -212,6 +212,51 @@ def test_pooled_fine_mass_is_block_mass_at_larger_size(factor):
     r = O.block_mass(q, k)
     np.testing.assert_allclose(pool_mass(r, factor), O.block_mass(q, k, block=B * factor),
                                atol=1e-13, rtol=0)
+
+def test_block_mass_16_pools_to_block_mass_32():
+    """Two by two 16-token blocks make one 32-token block: pooling the B = 16 masses
+    (factor 2) gives the B = 32 masses."""
+    from parity_utils import pool_mass
+    q, k, _ = rand_qkv(192, 8, 22, scale_q=2.0)
+    np.testing.assert_allclose(pool_mass(O.block_mass(q, k, block=16), 2), O.block_mass(q, k),
+                               atol=1e-13, rtol=0)
+
+
+def test_masked_attention_block16_brute_force():
+    """Scalar loops: row i attends j <= i with sel16[i // 16][j // 16]; an empty row gives
+    O = 0 and lse = -inf."""
+    n, d, scale = 64, 4, 0.5
+    q, k, v = rand_qkv(n, d, 23, scale_q=2.0)
+    rng = np.random.default_rng(23)
+    sel = np.tril(rng.random((4, 4)) < 0.5)
+    sel[2] = False                                   # rows 32..47 keep nothing
+    o, lse = O.masked_attention(q, k, v, sel, scale, block=16)
+    for i in range(n):
+        keep = [j for j in range(i + 1) if sel[i // 16][j // 16]]
+        if not keep:
+            assert np.all(o[i] == 0.0) and lse[i] == -np.inf
+            continue
+        logits = [scale * sum(q[i][c] * k[j][c] for c in range(d)) for j in keep]
+        mx = max(logits)
+        w = [math.exp(x - mx) for x in logits]
+        z = sum(w)
+        ref = [sum(w[t] * v[keep[t]][c] for t in range(len(keep))) / z for c in range(d)]
+        np.testing.assert_allclose(o[i], ref, atol=1e-13, rtol=0)
+        assert abs(lse[i] - (mx + math.log(z))) < 1e-12
+
+
+def test_masked_attention_block16_of_an_expanded_support_is_block32():
+    """A B = 16 support that keeps 2 x 2 subblocks exactly where a B = 32 support keeps a
+    block attends the same keys: identical results."""
+    q, k, v = rand_qkv(160, 8, 24, scale_q=2.0)
+    rng = np.random.default_rng(24)
+    sel32 = np.tril(rng.random((5, 5)) < 0.6)
+    np.fill_diagonal(sel32, True)
+    sel16 = np.repeat(np.repeat(sel32, 2, axis=0), 2, axis=1)
+    o16, l16 = O.masked_attention(q, k, v, sel16, block=16)
+    o32, l32 = O.masked_attention(q, k, v, sel32)
+    np.testing.assert_allclose(o16, o32, atol=1e-14, rtol=0)
+    np.testing.assert_allclose(l16, l32, atol=1e-14, rtol=0)
 
 def _element_mask_coarse(sel, factor, n):
     """Element (i, j) is attended iff j <= i and coarse block (i // 32f, j // 32f) is kept."""
