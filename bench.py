@@ -92,6 +92,19 @@ def dense_flops(cfg) -> float:
     return 4.0 * cfg.head_dim * cfg.bh * n * (n + 1) / 2
 
 
+def sparse_flops_b16(cfg, union16) -> float:
+    """4*d per admissible pair inside the kept 16-token blocks (16*16 off-diagonal,
+    16*17/2 diagonal), from the [BH, n/16, W] working-set words on the host."""
+    import numpy as np
+    n16 = cfg.seqlen // 16
+    words = union16.reshape(-1, n16, union16.shape[-1]).view(np.uint32)
+    bits = np.tril(np.unpackbits(words.view(np.uint8), axis=-1,
+                                 bitorder="little")[..., :n16].astype(bool))
+    diag = np.trace(bits, axis1=1, axis2=2).sum()
+    off = bits.sum() - diag
+    return 4.0 * cfg.head_dim * (off * 256 + diag * 136)
+
+
 def sparse_flops(cfg, row_offsets, col_idx) -> float:
     """4*d per admissible pair inside the scheduled blocks (32*32 off-diagonal, 32*33/2 diagonal)."""
     import numpy as np
@@ -226,7 +239,9 @@ class TrajectoryRunner:
         cfg = self.cfg
         nwin = cfg.window[1] - cfg.window[0] + 1
         # dense steps: 1 kernel; window steps: attention + mass + select; schedule: 3
-        return (cfg.t_d - nwin) + 3 * nwin + 3 + (cfg.steps - cfg.t_d)
+        # (block 16: 16-token mass + select; schedule fold + 3 + sub-masks = 5)
+        sched = 5 if self.block == 16 else 3
+        return (cfg.t_d - nwin) + 3 * nwin + sched + (cfg.steps - cfg.t_d)
 
     def run(self, q, k, v, events=None):
         """One trajectory.  If `events` is a dict, append (start, end) event pairs per call kind."""
@@ -239,6 +254,15 @@ class TrajectoryRunner:
             e.record()
             return e
 
+        if self.block == 16:   # the trajectory's own step calls, one event pair per step
+            for t in range(1, cfg.steps + 1):
+                a = ev() if events is not None else None
+                tr.step(t, q[t - 1], k[t - 1], v[t - 1], o=self.o)
+                if events is not None:
+                    kind = ("sparse" if t > cfg.t_d else
+                            "dense_mass" if tr.in_window(t) else "dense")
+                    events.setdefault(kind, []).append((a, ev()))
+            return self.o
         for t in range(1, cfg.steps + 1):
             qt, kt, vt = q[t - 1], k[t - 1], v[t - 1]
             if t <= cfg.t_d:
@@ -363,14 +387,20 @@ def cpu_oracle_sample(cfg, n_heads: int = 1, block: int = 32):
         O.causal_attention(q, k, v, cfg.scale)
         r = O.block_mass(q, k, cfg.scale, block=block)
         sup = O.select(r, cfg.eta)
-        if block != 32:
+        if block > 32:
             sup = O.expand_support(sup, block // 32)
         ro, ci = O.csr_schedule(sup)
         q, k, v = (bf16_bits_to_f64(x[i]) for x in steps[cfg.t_d + 1])
-        O.sparse_attention(q, k, v, ro, ci, cfg.scale)
         n = cfg.seqlen
         flops += 4.0 * cfg.head_dim * n * (n + 1) / 2
-        flops += sparse_flops(cfg.with_(batch=1, heads=1), ro, ci)
+        if block == 16:   # the oracle attends the 16-token support directly
+            O.masked_attention(q, k, v, sup, cfg.scale, block=16)
+            kept = np.tril(sup)
+            diag = int(np.trace(kept))
+            flops += 4.0 * cfg.head_dim * ((int(kept.sum()) - diag) * 256 + diag * 136)
+        else:
+            O.sparse_attention(q, k, v, ro, ci, cfg.scale)
+            flops += sparse_flops(cfg.with_(batch=1, heads=1), ro, ci)
     dt = time.perf_counter() - t0
     desc = (f"{len(heads)} head(s) of {cfg.name}: one dense exploration step with block mass and "
             f"eta-selection (B={block}), plus one block-sparse late step, numpy float64")
@@ -427,10 +457,13 @@ def bench_wise(args):
     ci = runner.traj.col_idx.cpu().numpy()
     nnz = int(ro[-1])
     f_dense = dense_flops(cfg)
-    f_sparse = sparse_flops(cfg, ro, ci)
+    if args.block == 16:
+        f_sparse = sparse_flops_b16(cfg, runner.traj.union.cpu().numpy())
+    else:
+        f_sparse = sparse_flops(cfg, ro, ci)
     nwin = cfg.window[1] - cfg.window[0] + 1
     traj_flops = cfg.t_d * f_dense + (cfg.steps - cfg.t_d) * f_sparse
-    density = nnz / (cfg.bh * cfg.nq * (cfg.nq + 1) / 2)
+    density = runner.traj.density()
 
     sampler = ClockSampler(local).start() if args.clocks else None
     barrier()
@@ -478,7 +511,8 @@ def bench_wise(args):
                 "traffic": profiled_traffic(kname, cfg.name),
                 "flops_per_launch": k_flops}
 
-    routing = routing_stats(cfg, q, k, v, device, args.block) if args.routing else None
+    routing = (routing_stats(cfg, q, k, v, device, args.block)
+               if args.routing and args.block != 16 else None)
 
     e2e = None
     if args.e2e:
@@ -506,7 +540,8 @@ def bench_wise(args):
                                f"{cfg.head_dim}, n={cfg.seqlen}, T={cfg.steps}, dense 1-{cfg.t_d}, "
                                f"union {cfg.window[0]}-{cfg.window[1]}, eta={cfg.eta}, "
                                f"B={args.block}"
-                               + (" (run as 32x32 subtiles)" if args.block != 32 else ""),
+                               + ({16: " (32x32 tiles with 16x16 sub-masks)", 32: ""}
+                                  .get(args.block, " (run as 32x32 subtiles)")),
                    "step": "one full WISE trajectory (dense + mass/select + schedule + sparse)",
                    "l2": "inputs larger than L2: every trajectory streams "
                          f"{3 * cfg.steps * cfg.bh * cfg.seqlen * cfg.head_dim * 2 / 1e9:.2f} GB "
@@ -517,7 +552,8 @@ def bench_wise(args):
         "late_step_iqr_us": [round(q25, 2), round(q75, 2)] if q25 is not None else None,
         "late_step_tflops": round(f_sparse / (sparse_us * 1e-6) / 1e12, 2) if sparse_us else None,
         "setup_inclusive_late_us": round(((cfg.steps - cfg.t_d) * sparse_us + sched_us)
-                                         / (cfg.steps - cfg.t_d), 2) if sparse_us else None,
+                                         / (cfg.steps - cfg.t_d), 2)
+                                   if sparse_us and sched_us else None,
         "dense_step_us": round(dense_us, 2) if dense_us else None,
         "dense_step_tflops": round(f_dense / (dense_us * 1e-6) / 1e12, 2) if dense_us else None,
         "window_step_us": round(dmass_us, 2) if dmass_us else None,
@@ -576,8 +612,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["wise", "reference"], default="wise")
     ap.add_argument("--config", default="4k")
-    ap.add_argument("--block", type=int, choices=[32, 64, 128], default=32,
-                    help="selection block size (64 / 128 run as 32x32 subtiles)")
+    ap.add_argument("--block", type=int, choices=[16, 32, 64, 128], default=32,
+                    help="selection block size (64 / 128 run as 32x32 subtiles, 16 as "
+                         "32x32 tiles with 16x16 sub-masks)")
     ap.add_argument("--eta", type=float, default=None,
                     help="mass threshold (default: the workload's, 0.95)")
     ap.add_argument("--t-d", dest="t_d", type=int, default=None,

@@ -10,7 +10,8 @@
  *                                  plus block mass on discovery-window steps)
  *                                wise_select_union     (cumulative-eta support,
  *                                  OR-ed into the working set; or
- *                                  wise_select_union_blocks for B = 64 / 128)
+ *                                  wise_select_union_blocks for B = 64 / 128;
+ *                                  the *_b16 calls for B = 16)
  *   once, after step t_d       : wise_build_schedule   (CSR key-block schedule)
  *   late steps t > t_d         : wise_sparse_attn      (block-sparse attention)
  *   analysis, off the hot path : wise_select_size_matched / _mass_matched
@@ -150,6 +151,49 @@ int wise_select_union(const float* mass, uint32_t* union_bits, uint32_t* step_bi
  */
 int wise_select_union_blocks(const float* mass, uint32_t* union_bits, uint32_t* step_bits,
                              float eta, int32_t block, wise_shape_t shape, void* stream);
+
+/*
+ * Block size 16 (WISE paper appendix C.6, "Block-Size Tradeoff": B in {16, 32, 64,
+ * 128}).  Selection runs on 16-token blocks; execution keeps 32 x 32 tiles, each
+ * carrying which of its four 16 x 16 sub-blocks are kept, so exactly the 16-token
+ * support is attended.  With n16 = seqlen / 16 and W16 = ceil(n16 / 32):
+ *
+ * wise_block_mass_b16: r[bh][q][b] = (1/16) sum over the 16 rows i of block q and the
+ *   keys j <= i of block b of exp(s_ij * scale - lse_i) (the block-mass equation of
+ *   section 5.1 at B = 16), for b <= q; entries b > q within the diagonal 32 x 32
+ *   block are written 0, the rest of b > q is not written.  QK^T is recomputed;
+ *   lse is the natural-log lse of wise_full_attn_mass.
+ *   q, k : bf16 [B, H, n, d] (k: [B, kv_heads, n, d]), 16-byte aligned;
+ *   lse  : fp32 [B, H, n];  mass16 : fp32 [B, H, n16, n16] output.
+ * wise_select_union_b16: wise_select_union over 16-token blocks: mass16 as above,
+ *   union16 / step16 uint32 [B, H, n16, W16] (same bit layout, OR-accumulated /
+ *   overwritten), same ranking, cut and eta rules.
+ * wise_build_schedule_b16: the CSR schedule over 32-token query and key blocks
+ *   (row_offsets [B*H*nq + 1], col_idx ascending per row, as wise_build_schedule)
+ *   listing key block b for query block q when any 16-block pair (2q + a, 2b + c),
+ *   a, c in {0, 1}, with 2b + c <= 2q + a is set in union16; sub[e] (uint8) holds
+ *   those four bits of entry e at bit 2a + c.  Workspace: device memory of
+ *   wise_schedule_b16_workspace_bytes(shape); capacity, nnz_out and errors as for
+ *   wise_build_schedule.
+ * wise_sparse_attn_b16: wise_sparse_attn where row i (16-row a = (i % 32) / 16)
+ *   attends key j of a listed block only if bit 2a + (j % 32) / 16 of the entry's
+ *   sub byte is set (and j <= i).  A row left with no key gets O = 0, lse = -inf.
+ *   An entry whose sub byte has no bit set is skipped.
+ * Errors: WISE_ERR_ARG (NULL pointers, eta <= 0, negative sizes), WISE_ERR_ALIGN,
+ *   WISE_ERR_SHAPE, WISE_ERR_WORKSPACE, WISE_ERR_CAPACITY, WISE_ERR_CUDA.
+ */
+int wise_block_mass_b16(const void* q, const void* k, const float* lse, float* mass16,
+                        wise_shape_t shape, void* stream);
+int wise_select_union_b16(const float* mass16, uint32_t* union16, uint32_t* step16, float eta,
+                          wise_shape_t shape, void* stream);
+size_t wise_schedule_b16_workspace_bytes(wise_shape_t shape);
+int wise_build_schedule_b16(const uint32_t* union16, int32_t* row_offsets, int32_t* col_idx,
+                            uint8_t* sub, int64_t col_capacity, int64_t* nnz_out,
+                            void* workspace, size_t workspace_bytes, wise_shape_t shape,
+                            void* stream);
+int wise_sparse_attn_b16(const void* q, const void* k, const void* v, void* o,
+                         const int32_t* row_offsets, const int32_t* col_idx, const uint8_t* sub,
+                         int64_t col_count, float* lse, wise_shape_t shape, void* stream);
 
 /*
  * Selection-only controls (WISE paper appendix B, "Intervention controls").  Both

@@ -51,6 +51,14 @@ _SIGNATURES = {
     "wise_select_union": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_float, WiseShape, _vp]),
     "wise_select_union_blocks": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_float, ctypes.c_int32,
                                                 WiseShape, _vp]),
+    "wise_block_mass_b16": (ctypes.c_int, [_vp, _vp, _vp, _vp, WiseShape, _vp]),
+    "wise_select_union_b16": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_float, WiseShape, _vp]),
+    "wise_schedule_b16_workspace_bytes": (ctypes.c_size_t, [WiseShape]),
+    "wise_build_schedule_b16": (ctypes.c_int, [_vp, _vp, _vp, _vp, ctypes.c_int64,
+                                               ctypes.POINTER(ctypes.c_int64), _vp,
+                                               ctypes.c_size_t, WiseShape, _vp]),
+    "wise_sparse_attn_b16": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int64,
+                                            _vp, WiseShape, _vp]),
     "wise_select_size_matched": (ctypes.c_int, [_vp, _vp, _vp, WiseShape, _vp]),
     "wise_select_mass_matched": (ctypes.c_int, [_vp, _vp, _vp, WiseShape, _vp]),
     "wise_support_mass": (ctypes.c_int, [_vp, _vp, _vp, WiseShape, _vp]),

@@ -370,6 +370,112 @@ int wise_sparse_attn(const void* q, const void* k, const void* v, void* o,
   return ok();
 }
 
+// ------------------------------------------------------------- block size 16
+
+int wise_block_mass_b16(const void* q, const void* k, const float* lse, float* mass16,
+                        wise_shape_t shape, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!q || !k || !lse || !mass16) return fail(WISE_ERR_ARG, "q, k, lse and mass16 must be non-NULL");
+  if (!aligned16(q) || !aligned16(k)) return fail(WISE_ERR_ALIGN, "q, k must be 16-byte aligned");
+  wise::AttnParams pm{};
+  pm.lse_in = lse;
+  pm.mass = mass16;
+  pm.fine16 = 1;
+  rc = launch_attn(wise::kModeMass, q, k, nullptr, nullptr, pm, shape, stream);
+  if (rc) return rc;
+  return ok();
+}
+
+int wise_select_union_b16(const float* mass16, uint32_t* union16, uint32_t* step16, float eta,
+                          wise_shape_t shape, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!mass16 || !union16) return fail(WISE_ERR_ARG, "mass16 and union16 must be non-NULL");
+  if (!(eta > 0.f)) return fail(WISE_ERR_ARG, "eta must be > 0 (got %g)", (double)eta);
+  cudaError_t e = wise::launch_select_union(mass16, union16, step16, eta,
+                                            shape.batch * shape.heads, shape.seqlen / 16,
+                                            static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "select_union_b16 launch");
+  return ok();
+}
+
+static size_t b16_bits32_offset(long long rows) {
+  return (wise::schedule_workspace_bytes(rows) + 255) & ~(size_t)255;
+}
+
+size_t wise_schedule_b16_workspace_bytes(wise_shape_t shape) {
+  if (check_shape(shape)) return 0;
+  const long long nq = shape.seqlen / 32;
+  const long long rows = (long long)shape.batch * shape.heads * nq;
+  return b16_bits32_offset(rows) + (size_t)rows * ((nq + 31) / 32) * sizeof(uint32_t);
+}
+
+int wise_build_schedule_b16(const uint32_t* union16, int32_t* row_offsets, int32_t* col_idx,
+                            uint8_t* sub, int64_t col_capacity, int64_t* nnz_out,
+                            void* workspace, size_t workspace_bytes, wise_shape_t shape,
+                            void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!union16 || !row_offsets || !col_idx || !sub)
+    return fail(WISE_ERR_ARG, "union16, row_offsets, col_idx and sub must be non-NULL");
+  if (col_capacity < 0) return fail(WISE_ERR_ARG, "col_capacity must be >= 0");
+  const long long nq = shape.seqlen / 32;
+  const long long rows = (long long)shape.batch * shape.heads * nq;
+  const long long max_nnz = rows * (nq + 1) / 2;
+  if (max_nnz > 0x7fffffffll) return fail(WISE_ERR_SHAPE, "schedule may exceed 2^31 entries");
+  const size_t need = wise_schedule_b16_workspace_bytes(shape);
+  if (!workspace || workspace_bytes < need)
+    return fail(WISE_ERR_WORKSPACE, "workspace of %zu bytes required", need);
+  if (!nnz_out && col_capacity < max_nnz)
+    return fail(WISE_ERR_CAPACITY,
+                "col_capacity %lld < worst case %lld; pass nnz_out to check the exact size",
+                (long long)col_capacity, max_nnz);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* bits32 =
+      reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + b16_bits32_offset(rows));
+  const int BH = shape.batch * shape.heads;
+  cudaError_t e = wise::launch_fold16(union16, bits32, BH, (int)nq, st);
+  if (e == cudaSuccess)
+    e = wise::launch_build_schedule(bits32, row_offsets, col_idx, col_capacity, workspace, rows,
+                                    (int)nq, st);
+  if (e == cudaSuccess)
+    e = wise::launch_sub16(union16, row_offsets, col_idx, sub, col_capacity, BH, (int)nq, st);
+  if (e != cudaSuccess) return cuda_fail(e, "build_schedule_b16 launch");
+  if (nnz_out) {
+    int32_t nnz = 0;
+    e = cudaMemcpyAsync(&nnz, row_offsets + rows, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "reading nnz");
+    *nnz_out = nnz;
+    if (nnz > col_capacity)
+      return fail(WISE_ERR_CAPACITY, "schedule has %d entries, capacity %lld", nnz,
+                  (long long)col_capacity);
+  }
+  return ok();
+}
+
+int wise_sparse_attn_b16(const void* q, const void* k, const void* v, void* o,
+                         const int32_t* row_offsets, const int32_t* col_idx, const uint8_t* sub,
+                         int64_t col_count, float* lse, wise_shape_t shape, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !row_offsets || ((!col_idx || !sub) && col_count > 0))
+    return fail(WISE_ERR_ARG, "q, k, v, o, row_offsets, col_idx, sub must be non-NULL");
+  if (col_count < 0) return fail(WISE_ERR_ARG, "col_count must be >= 0");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(WISE_ERR_ALIGN, "q, k, v, o must be 16-byte aligned");
+  wise::AttnParams p{};
+  p.lse = lse;
+  p.row_offsets = row_offsets;
+  p.col_idx = col_idx;
+  p.sub = sub;
+  p.col_count = col_count;
+  rc = launch_attn(wise::kModeSparse16, q, k, v, o, p, shape, stream);
+  if (rc) return rc;
+  return ok();
+}
+
 int wise_device_status(uint32_t* status_out, int clear) {
   if (!status_out) return fail(WISE_ERR_ARG, "status_out must be non-NULL");
   cudaError_t e = cudaDeviceSynchronize();

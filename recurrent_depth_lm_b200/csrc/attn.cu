@@ -79,7 +79,9 @@ struct Cfg {
   static constexpr int kPanels = (D + 63) / 64;
   static constexpr bool kAttn = MODE != kModeMass;
   static constexpr int kTileBytes = kPanels * kPanelBytes;  // Q tile, one K or V stage
-  static constexpr int kKStages = kAttn ? (D <= 64 ? 4 : 3) : (D <= 64 ? 6 : 4);
+  // block-size-16 sparse mode: its sub-mask planes need the shared memory of one K stage
+  static constexpr int kKStages =
+      kAttn ? (D <= 64 ? 4 : (MODE == kModeSparse16 ? 2 : 3)) : (D <= 64 ? 6 : 4);
   static constexpr int kVStages = kAttn ? (D <= 64 ? 4 : 2) : 0;
   static constexpr int kVRing = kVStages > 0 ? kVStages : 1;  // barrier slots (mass mode: unused)
   static constexpr int kOffQ = 0;
@@ -87,7 +89,9 @@ struct Cfg {
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
   static constexpr int kOffEnt = kOffV + kVStages * kTileBytes;
   static constexpr int kOffMask = kOffEnt + 2 * kRing * (int)sizeof(Entry);
-  static constexpr int kOffBar = kOffMask + 2 * 4 * kMaxWords * 4;
+  // per slot: 4 row masks of kMaxWords words; sparse16 adds 16 sub-mask planes
+  static constexpr int kMaskWords = (MODE == kModeSparse16 ? 20 : 4) * kMaxWords;
+  static constexpr int kOffBar = kOffMask + 2 * kMaskWords * 4;
   // q_full[2], q_empty[2], k_full[K], k_empty[K], v_full[V], v_empty[V], e_full[2][R],
   // e_empty[2][R], s_full[2], s_free[2], p_full[2], o_done[2], o_free[2], final
   static constexpr int kNumBars = 4 + 2 * kKStages + 2 * kVRing + 4 * kRing + 11;
@@ -157,6 +161,20 @@ struct MaskList {
       if ((mask[r * kMaxWords + w] >> bit) & 1u) own |= 1 << r;
     return true;
   }
+  // Block size 16: own = the 16 sub-mask bits (row r, bit j) at bit 4 r + j, read from
+  // the planes by lanes 0..15 at once (whole warp, converged).
+  __device__ bool pop_sub(int& kb, int& own, int lane) {
+    while (cur == 0) {
+      if (++w >= words) return false;
+      cur = mask[w] | mask[kMaxWords + w] | mask[2 * kMaxWords + w] | mask[3 * kMaxWords + w];
+    }
+    const int bit = __ffs(cur) - 1;
+    cur &= cur - 1;
+    kb = w * 32 + bit;
+    const bool set = lane < 16 && ((mask[(4 + lane) * kMaxWords + w] >> bit) & 1u);
+    own = (int)(__ballot_sync(0xffffffffu, set) & 0xffffu);
+    return true;
+  }
 };
 
 // Build the 4 per-row bitmasks of a sparse tile (whole producer warp).  The tile's
@@ -164,9 +182,14 @@ struct MaskList {
 // [0, col_count], one strided pass over col_idx[row_offsets[r0], row_offsets[r0 + nr])
 // covers them.  Otherwise each row is taken on its own and a row with bad offsets
 // is dropped.  Entries outside [0, q] are dropped.  Anything dropped is flagged.
+//
+// Block size 16 (kSub): entry e also carries p.sub[e], bit 2a + c = 16-row a of the
+// query block keeps 16-column half c of the key block.  Bit j of row r goes to plane
+// 4 r + j (mask + (4 + 4 r + j) * kMaxWords); an entry with no bit set is dropped.
+template <bool kSub>
 __device__ void build_tile_masks(uint32_t* mask, const AttnParams& p, int bh, int Qt, int lane) {
   const int words = (p.nq + 31) / 32;
-  for (int x = lane; x < 4 * kMaxWords; x += 32) mask[x] = 0u;
+  for (int x = lane; x < (kSub ? 20 : 4) * kMaxWords; x += 32) mask[x] = 0u;
   const int qb0 = Qt * 4;
   const int nr = min(4, p.nq - qb0);                 // rows of this tile
   const long long row0 = (long long)bh * p.nq + qb0;
@@ -186,10 +209,12 @@ __device__ void build_tile_masks(uint32_t* mask, const AttnParams& p, int bh, in
     // 8 entries per lane per round: all loads are issued before any is used
     for (long long e0 = beg + lane; e0 < end; e0 += 8 * 32) {
       int kbs[8];
+      uint32_t subs[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const long long e = e0 + u * 32;
         kbs[u] = e < end ? p.col_idx[e] : 0;
+        subs[u] = (kSub && e < end) ? (uint32_t)p.sub[e] & 15u : 15u;
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -197,10 +222,17 @@ __device__ void build_tile_masks(uint32_t* mask, const AttnParams& p, int bh, in
         if (e >= end) break;
         const int r = (e >= o1) + (e >= o2) + (e >= o3);   // row of entry e
         const int kb = kbs[u];
-        if (kb >= 0 && kb <= qb0 + r && kb < words * 32)
-          atomicOr(&mask[r * kMaxWords + (kb >> 5)], 1u << (kb & 31));
-        else
+        if (kb >= 0 && kb <= qb0 + r && kb < words * 32) {
+          if (subs[u] != 0u) atomicOr(&mask[r * kMaxWords + (kb >> 5)], 1u << (kb & 31));
+          if (kSub) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              if ((subs[u] >> j) & 1u)
+                atomicOr(&mask[(4 + 4 * r + j) * kMaxWords + (kb >> 5)], 1u << (kb & 31));
+          }
+        } else {
           bad = true;
+        }
       }
     }
   } else {
@@ -212,8 +244,15 @@ __device__ void build_tile_masks(uint32_t* mask, const AttnParams& p, int bh, in
       const int qb = qb0 + r;
       for (long long e = beg + lane; e < end; e += 32) {
         const int kb = p.col_idx[e];
-        if (kb >= 0 && kb <= qb && kb < words * 32)
+        const uint32_t sb = kSub ? (uint32_t)p.sub[e] & 15u : 15u;
+        if (kb >= 0 && kb <= qb && kb < words * 32 && sb != 0u) {
           atomicOr(&mask[r * kMaxWords + (kb >> 5)], 1u << (kb & 31));
+          if (kSub) {
+            for (int j = 0; j < 4; ++j)
+              if ((sb >> j) & 1u)
+                atomicOr(&mask[(4 + 4 * r + j) * kMaxWords + (kb >> 5)], 1u << (kb & 31));
+          }
+        }
       }
     }
   }
@@ -227,6 +266,14 @@ template <int N>
 __device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
 #pragma unroll
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+// Block size 16: scores of the 16-column halves a row does not keep become -inf
+// (keep bit c = columns 16 c .. 16 c + 15).
+__device__ __forceinline__ void half_mask(uint32_t (&v)[32], uint32_t keep) {
+#pragma unroll
+  for (int c = 0; c < 32; ++c)
+    if (!((keep >> (c >> 4)) & 1u)) v[c] = __float_as_uint(-INFINITY);
 }
 
 // kb[s] of a 4-entry register array for a runtime s, without local memory.
@@ -292,7 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sK = smem_u32(smem + C::kOffK);
   const uint32_t sV = smem_u32(smem + C::kOffV);
   Entry* ents = (Entry*)(smem + C::kOffEnt);               // [2][kRing]
-  uint32_t* masks = (uint32_t*)(smem + C::kOffMask);       // [2][4][kMaxWords]
+  uint32_t* masks = (uint32_t*)(smem + C::kOffMask);       // [2][kMaskWords]
+  constexpr bool kSparseAny = MODE == kModeSparse || MODE == kModeSparse16;
   const uint32_t bar0 = smem_u32(smem + C::kOffBar);
   auto bar_q_full = [&](int x) { return bar0 + 8 * x; };
   auto bar_q_empty = [&](int x) { return bar0 + 16 + 8 * x; };
@@ -393,9 +441,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         decode_tile(tile, p.BH, ntq, S.bh, S.qt);
         S.kvh = S.bh / p.group;
-        if (MODE == kModeSparse) {
-          uint32_t* msk = masks + X * 4 * kMaxWords;
-          build_tile_masks(msk, p, S.bh, S.qt, lane);
+        if (kSparseAny) {
+          uint32_t* msk = masks + X * C::kMaskWords;
+          build_tile_masks<MODE == kModeSparse16>(msk, p, S.bh, S.qt, lane);
           S.ml.init(msk, (p.nq + 31) / 32);
         } else {
           S.dl.init(S.qt, p.nq);
@@ -417,7 +465,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int n = 0;
       {
         int kb, own;
-        while (n < kSlots && (MODE == kModeSparse ? S.ml.pop(kb, own) : S.dl.pop(kb, own))) {
+        while (n < kSlots && (MODE == kModeSparse16 ? S.ml.pop_sub(kb, own, lane)
+                              : MODE == kModeSparse ? S.ml.pop(kb, own)
+                                                    : S.dl.pop(kb, own))) {
           kbv[n] = kb;
           ownv[n] = own;
           ++n;
@@ -428,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ownv[0] = 0;
         n = 1;
       }
-      const bool last = (MODE == kModeSparse) ? S.ml.empty() : S.dl.empty();
+      const bool last = kSparseAny ? S.ml.empty() : S.dl.empty();
       const int ks = g % NK;
       if (g >= (uint32_t)NK &&
           !warp_wait(bar_k_empty(ks), ((g / NK) - 1) & 1, abort_flag, p.status))
@@ -701,6 +751,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int ns = e.ns;
         uint32_t vmask = 0u, dmask = 0u;   // key blocks this row sees; diagonal blocks
+        uint32_t hmask = 0u;               // block size 16: kept halves, 2 bits per block
         if (first) {
           bh = e.bh;
           qb = e.Qt * 4 + qw;
@@ -710,7 +761,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int s = 0; s < kSlots; ++s) {
-          if (s < ns && ((e.own[s] >> qw) & 1)) {
+          if (MODE == kModeSparse16) {
+            // own: bit 4 r + 2 a + c = 16-row a of query block r keeps half c
+            const int o4 = s < ns ? (e.own[s] >> (4 * qw)) & 15 : 0;
+            if (o4 != 0) {
+              vmask |= 1u << s;
+              if (e.kb[s] == qb) dmask |= 1u << s;
+              hmask |= (uint32_t)((o4 >> (2 * (lane >> 4))) & 3) << (2 * s);
+            }
+          } else if (s < ns && ((e.own[s] >> qw) & 1)) {
             vmask |= 1u << s;
             if (e.kb[s] == qb) dmask |= 1u << s;
           }
@@ -731,8 +790,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32(t_lane + s_col + s * 32, v);
             tmem_wait_ld();
             reg_fence(v);
-            float a4[4] = {0.f, 0.f, 0.f, 0.f};
             const bool diag = (dmask >> s) & 1u;
+            if (p.fine16) {
+              // 16-token blocks: lanes 0..15 / 16..31 are 16-rows 2 qb / 2 qb + 1; a4[0..1]
+              // would mix the halves, so sum each 16-column half on its own
+              float lo = 0.f, hi = 0.f;
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                const float ev = fast_exp2(fmaf(__uint_as_float(v[c]), sl2, -lse_l2));
+                const float x = (diag && c > lane) ? 0.f : ev;
+                if (c < 16) lo += x; else hi += x;
+              }
+#pragma unroll
+              for (int o = 8; o > 0; o >>= 1) {
+                lo += __shfl_xor_sync(0xffffffffu, lo, o);
+                hi += __shfl_xor_sync(0xffffffffu, hi, o);
+              }
+              if ((lane & 15) == 0) {
+                const long long nq16 = 2ll * p.nq;
+                float* dst = p.mass + ((long long)bh * nq16 + 2 * qb + (lane >> 4)) * nq16 +
+                             2 * e.kb[s];
+                dst[0] = lo * (1.0f / 16.0f);
+                dst[1] = hi * (1.0f / 16.0f);
+              }
+              continue;
+            }
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
               const float ev = fast_exp2(fmaf(__uint_as_float(v[c]), sl2, -lse_l2));
@@ -774,6 +857,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < 32; ++c)
                   if (c > lane) sr[h][c] = __float_as_uint(-INFINITY);
               }
+              if (MODE == kModeSparse16 && ((hmask >> (2 * (s0 + h))) & 3u) != 3u)
+                half_mask(sr[h], (hmask >> (2 * (s0 + h))) & 3u);
 #pragma unroll
               for (int c = 0; c < 32; c += 8) {
 #pragma unroll
@@ -806,6 +891,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int c = 0; c < 32; ++c)
                 if (c > lane) v[c] = __float_as_uint(-INFINITY);
             }
+            if (MODE == kModeSparse16 && ((hmask >> (2 * s)) & 3u) != 3u)
+              half_mask(v, (hmask >> (2 * s)) & 3u);
             uint64_t rs2[2] = {0ull, 0ull};
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
@@ -941,6 +1028,7 @@ cudaError_t launch_attention(int mode, int d, const CUtensorMap& tq, const CUten
     case kModeDense: return launch_mode<kModeDense>(d, tq, tk, tv, p, grid, stream, why);
     case kModeSparse: return launch_mode<kModeSparse>(d, tq, tk, tv, p, grid, stream, why);
     case kModeMass: return launch_mode<kModeMass>(d, tq, tk, tv, p, grid, stream, why);
+    case kModeSparse16: return launch_mode<kModeSparse16>(d, tq, tk, tv, p, grid, stream, why);
   }
   return cudaErrorInvalidValue;
 }
@@ -951,6 +1039,11 @@ int attention_smem_bytes(int mode, int d) {
     if (d == 64) return pick(Cfg<64, kModeMass>{});
     if (d == 96) return pick(Cfg<96, kModeMass>{});
     return pick(Cfg<128, kModeMass>{});
+  }
+  if (mode == kModeSparse16) {
+    if (d == 64) return pick(Cfg<64, kModeSparse16>{});
+    if (d == 96) return pick(Cfg<96, kModeSparse16>{});
+    return pick(Cfg<128, kModeSparse16>{});
   }
   if (d == 64) return pick(Cfg<64, kModeDense>{});
   if (d == 96) return pick(Cfg<96, kModeDense>{});

@@ -195,6 +195,8 @@ cudaError_t launch_select_union(const float* mass, uint32_t* union_bits, uint32_
     select_union_kernel<8><<<grid, block, 0, stream>>>(mass, union_bits, step_bits, eta, rows, nq);
   else if (W <= 16)
     select_union_kernel<16><<<grid, block, 0, stream>>>(mass, union_bits, step_bits, eta, rows, nq);
+  else if (W <= 32)  // 16-token blocks at n = 16384
+    select_union_kernel<32><<<grid, block, 0, stream>>>(mass, union_bits, step_bits, eta, rows, nq);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();

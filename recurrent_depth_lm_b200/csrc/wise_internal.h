@@ -9,7 +9,9 @@
 
 namespace wise {
 
-enum { kModeDense = 0, kModeSparse = 1, kModeMass = 2 };
+// kModeSparse16: block-sparse attention whose 32 x 32 blocks carry 16 x 16 sub-masks
+// (block size 16).
+enum { kModeDense = 0, kModeSparse = 1, kModeMass = 2, kModeSparse16 = 3 };
 
 struct AttnParams {
   int BH;               // batch * heads
@@ -21,11 +23,13 @@ struct AttnParams {
   void* o;              // [BH, n, d] bf16 output (dense / sparse)
   float* lse;           // [BH, n] output (dense / sparse), nullable
   const float* lse_in;  // [BH, n] input (mass mode)
-  float* mass;          // [BH, nq, nq] output (mass mode)
+  float* mass;          // [BH, nq, nq] output (mass mode); [BH, 2nq, 2nq] when fine16
+  int fine16;           // mass mode: block mass of 16-token blocks
   float* blse;          // [BH, nq, n] block log2-sum-exp side output (dense mode), nullable
   const int32_t* row_offsets;  // sparse mode
   const int32_t* col_idx;      // sparse mode
   long long col_count;         // sparse mode: valid entries of col_idx
+  const uint8_t* sub;          // sparse16 mode: 16 x 16 sub-mask bits of each col_idx entry
   unsigned int* status;        // device status word
 };
 
@@ -56,6 +60,15 @@ cudaError_t launch_select_control(const float* mass, const uint32_t* ref_bits, u
 // retained[bh * nq + q] = sum of mass over the set admissible bits of the row.
 cudaError_t launch_support_mass(const float* mass, const uint32_t* bits, float* retained, int BH,
                                 int nq, cudaStream_t stream);
+
+// Block size 16: fold the [BH, 2nq, W16] 16-token masks into 32-token rows [BH, nq, W]
+// (a 32-block is kept if any of its four 16-blocks is, causally), then the sub-mask of
+// every schedule entry: bit 2a + c = 16-row 2q + a keeps 16-block 2b + c.
+cudaError_t launch_fold16(const uint32_t* union16, uint32_t* bits32, int BH, int nq,
+                          cudaStream_t stream);
+cudaError_t launch_sub16(const uint32_t* union16, const int32_t* row_offsets,
+                         const int32_t* col_idx, uint8_t* sub, long long capacity, int BH,
+                         int nq, cudaStream_t stream);
 
 size_t schedule_workspace_bytes(long long rows);
 cudaError_t launch_build_schedule(const uint32_t* union_bits, int32_t* row_offsets,

@@ -189,6 +189,83 @@ def sparse_attn(q, k, v, row_offsets, col_idx, col_count: int | None = None, *, 
     return o, lse
 
 
+# ------------------------------------------------------------------ block size 16
+
+def block_mass_b16(q, k, lse, *, out=None, scale=None, stream=None):
+    """Block mass of 16-token blocks from the dense pass's lse: fp32 [B, H, n/16, n/16]."""
+    b, h, n, _ = q.shape
+    if out is None:
+        out = torch.empty(b, h, n // 16, n // 16, dtype=torch.float32, device=q.device)
+    kv = _check_qkv(q, k, k, q)
+    rc = lib.wise_block_mass_b16(_ptr(q), _ptr(k), _ptr(lse), _ptr(out), shape_of(q, scale, kv),
+                                 _stream(stream))
+    check(rc, "wise_block_mass_b16")
+    return out
+
+
+def new_bitmask_b16(b: int, h: int, n: int, device) -> torch.Tensor:
+    """Zeroed 16-token working-set masks [B, H, n/16, ceil(n/16/32)]."""
+    return new_bitmask(b, h, n // 16, device)
+
+
+def select_union_b16(mass16, union16, eta: float, *, step_bits=None, head_dim: int = 128,
+                     stream=None):
+    """OR the cumulative-eta support over 16-token blocks into `union16` (in place)."""
+    b, h, n16, _ = mass16.shape
+    if mass16.dtype != torch.float32 or union16.dtype != torch.int32:
+        raise ValueError("mass16 must be float32 and union16 int32 (uint32 bit patterns)")
+    rc = lib.wise_select_union_b16(_ptr(mass16), _ptr(union16), _ptr(step_bits), float(eta),
+                                   WiseShape(b, h, n16 * 16, head_dim, 0.0), _stream(stream))
+    check(rc, "wise_select_union_b16")
+    return union16
+
+
+def schedule_b16_workspace(b: int, h: int, n: int, head_dim: int, device) -> torch.Tensor:
+    nbytes = lib.wise_schedule_b16_workspace_bytes(WiseShape(b, h, n, head_dim, 0.0))
+    return torch.empty(max(1, nbytes), dtype=torch.uint8, device=device)
+
+
+def build_schedule_b16(union16, *, head_dim: int = 128, row_offsets=None, col_idx=None,
+                       sub=None, workspace=None, exact_nnz: bool = True, stream=None):
+    """32-token CSR schedule plus 16 x 16 sub-masks.  Returns (row_offsets, col_idx, sub, nnz)."""
+    b, h, n16, _ = union16.shape
+    n = n16 * 16
+    nq = n // BLOCK
+    dev = union16.device
+    if row_offsets is None:
+        row_offsets = torch.empty(b * h * nq + 1, dtype=torch.int32, device=dev)
+    if col_idx is None:
+        col_idx = torch.empty(schedule_max_nnz(b, h, n, head_dim), dtype=torch.int32, device=dev)
+    if sub is None:
+        sub = torch.empty(col_idx.numel(), dtype=torch.uint8, device=dev)
+    if sub.numel() < col_idx.numel():
+        raise ValueError("sub must hold one byte per col_idx entry")
+    if workspace is None:
+        workspace = schedule_b16_workspace(b, h, n, head_dim, dev)
+    nnz = ctypes.c_int64(-1)
+    rc = lib.wise_build_schedule_b16(_ptr(union16), _ptr(row_offsets), _ptr(col_idx), _ptr(sub),
+                                     col_idx.numel(), ctypes.byref(nnz) if exact_nnz else None,
+                                     _ptr(workspace), workspace.numel(),
+                                     WiseShape(b, h, n, head_dim, 0.0), _stream(stream))
+    check(rc, "wise_build_schedule_b16")
+    return row_offsets, col_idx, sub, (int(nnz.value) if exact_nnz else None)
+
+
+def sparse_attn_b16(q, k, v, row_offsets, col_idx, sub, col_count: int | None = None, *,
+                    o=None, lse=None, scale=None, stream=None):
+    """Block-sparse causal attention whose entries carry 16 x 16 sub-masks.  Returns (o, lse)."""
+    if o is None:
+        o = torch.empty_like(q)
+    kv = _check_qkv(q, k, v, o)
+    if col_count is None:
+        col_count = col_idx.numel()
+    rc = lib.wise_sparse_attn_b16(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(row_offsets),
+                                  _ptr(col_idx), _ptr(sub), int(col_count), _ptr(lse),
+                                  shape_of(q, scale, kv), _stream(stream))
+    check(rc, "wise_sparse_attn_b16")
+    return o, lse
+
+
 def device_status(clear: bool = True) -> int:
     st = ctypes.c_uint32(0)
     check(lib.wise_device_status(ctypes.byref(st), 1 if clear else 0), "wise_device_status")

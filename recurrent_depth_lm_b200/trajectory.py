@@ -7,7 +7,9 @@ select each query block's cumulative-eta key-block support and union it;
 after step t_d the union is compacted once into a CSR schedule; every later
 step runs block-sparse attention over that schedule with fresh Q, K, V.
 Appendix C.6's block-size variants (block = 64 or 128) select on coarser blocks
-and run the result as exact 32 x 32 subtiles.
+and run the result as exact 32 x 32 subtiles; block = 16 selects on 16-token
+blocks (masses recomputed from the dense pass's lse) and runs 32 x 32 tiles that
+carry 16 x 16 sub-masks.
 
 The selection-only controls of appendix B ("Intervention controls") replace the
 frozen support: "static95" is the eta-support of step 1 alone, "size_matched"
@@ -40,8 +42,10 @@ class WiseTrajectory:
             raise ValueError(f"support must be one of {SUPPORTS}")
         if support in ("size_matched", "mass_matched") and block != ops.BLOCK:
             raise ValueError("the size- and mass-matched controls are defined for block = 32")
-        if block not in (32, 64, 128):
-            raise ValueError("block must be 32, 64 or 128")
+        if block not in (16, 32, 64, 128):
+            raise ValueError("block must be 16, 32, 64 or 128")
+        if block == 16 and (support != "wise" or track_retained):
+            raise ValueError("block 16 runs the WISE support without retained-mass tracking")
         if seqlen % block:
             raise ValueError(f"seqlen must be a multiple of the block size {block}")
         self.block = block
@@ -53,6 +57,11 @@ class WiseTrajectory:
         self.lse = torch.empty(batch, heads, seqlen, dtype=torch.float32, device=dev)
         self.mass = torch.empty(batch, heads, self.nq, self.nq, dtype=torch.float32, device=dev)
         self.union = ops.new_bitmask(batch, heads, self.nq, dev)
+        self.mass16 = self.sub = self.ws16 = None
+        if block == 16:   # 16-token masses and working set; sub-masks of the schedule
+            self.mass16 = torch.empty(batch, heads, seqlen // 16, seqlen // 16,
+                                      dtype=torch.float32, device=dev)
+            self.union = ops.new_bitmask_b16(batch, heads, seqlen, dev)
         # per-(row, key block) log-sum-exps of the one-pass block mass (window steps)
         self.mass_ws = ops.mass_workspace(batch, heads, seqlen, head_dim, dev)
         self.step_bits = {}
@@ -61,6 +70,9 @@ class WiseTrajectory:
         self.col_idx = torch.empty(ops.schedule_max_nnz(batch, heads, seqlen, head_dim),
                                    dtype=torch.int32, device=dev)
         self.workspace = ops.schedule_workspace(batch, heads, seqlen, head_dim, dev)
+        if block == 16:
+            self.sub = torch.empty(self.col_idx.numel(), dtype=torch.uint8, device=dev)
+            self.workspace = ops.schedule_b16_workspace(batch, heads, seqlen, head_dim, dev)
         self.scheduled = False
         self.support = support
         # step-1 block masses and the control support (selection-only controls)
@@ -93,7 +105,18 @@ class WiseTrajectory:
         """Attention of recurrent step t (1-based).  Returns O."""
         if t <= self.t_d:
             first = t == 1 and self.mass1 is not None   # step-1 masses for the controls
-            if self.in_window(t) or first:
+            if self.block == 16 and self.in_window(t):
+                o, _, _ = ops.full_attn_mass(q, k, v, o=o, lse=self.lse, scale=self.scale,
+                                             stream=stream)
+                ops.block_mass_b16(q, k, self.lse, out=self.mass16, scale=self.scale,
+                                   stream=stream)
+                sb = None
+                if self.keep_step_bits:
+                    sb = torch.empty_like(self.union)
+                    self.step_bits[t] = sb
+                ops.select_union_b16(self.mass16, self.union, self.eta, step_bits=sb,
+                                     head_dim=self.d, stream=stream)
+            elif self.in_window(t) or first:
                 m = self.mass1 if first else self.mass
                 o, _, _ = ops.full_attn_mass(q, k, v, o=o, lse=self.lse, mass=m,
                                              workspace=self.mass_ws, scale=self.scale,
@@ -116,8 +139,14 @@ class WiseTrajectory:
             return o
         if not self.scheduled:
             raise RuntimeError("late step before the schedule was built (t <= t_d never reached)")
-        o, _ = ops.sparse_attn(q, k, v, self.row_offsets, self.col_idx, self.col_idx.numel(),
-                               o=o, lse=lse, scale=self.scale, stream=stream)
+        if self.block == 16:
+            o, _ = ops.sparse_attn_b16(q, k, v, self.row_offsets, self.col_idx, self.sub,
+                                       self.col_idx.numel(), o=o, lse=lse, scale=self.scale,
+                                       stream=stream)
+        else:
+            o, _ = ops.sparse_attn(q, k, v, self.row_offsets, self.col_idx,
+                                   self.col_idx.numel(), o=o, lse=lse, scale=self.scale,
+                                   stream=stream)
         if self.track_retained:
             ops.full_attn_mass(q, k, v, o=self.o_scratch, lse=self.lse, mass=self.mass,
                                workspace=self.mass_ws, scale=self.scale, stream=stream)
@@ -132,9 +161,14 @@ class WiseTrajectory:
         elif self.support == "mass_matched":
             ops.select_mass_matched(self.mass1, self.union, out=self.control, head_dim=self.d,
                                     stream=stream)
-        ops.build_schedule(self.frozen, head_dim=self.d, row_offsets=self.row_offsets,
-                           col_idx=self.col_idx, workspace=self.workspace, exact_nnz=False,
-                           stream=stream)
+        if self.block == 16:
+            ops.build_schedule_b16(self.union, head_dim=self.d, row_offsets=self.row_offsets,
+                                   col_idx=self.col_idx, sub=self.sub, workspace=self.workspace,
+                                   exact_nnz=False, stream=stream)
+        else:
+            ops.build_schedule(self.frozen, head_dim=self.d, row_offsets=self.row_offsets,
+                               col_idx=self.col_idx, workspace=self.workspace, exact_nnz=False,
+                               stream=stream)
         self.scheduled = True
 
     def retained_future_mass(self) -> float:
@@ -147,5 +181,12 @@ class WiseTrajectory:
         return int(self.row_offsets[-1].item())
 
     def density(self) -> float:
-        """Fraction of admissible (causal) query-key blocks retained."""
-        return self.nnz() / (self.b * self.h * self.nq * (self.nq + 1) / 2)
+        """Fraction of admissible (causal) query-key blocks retained, counted at the
+        selection's block size (16-token blocks for block = 16)."""
+        if self.block != 16:
+            return self.nnz() / (self.b * self.h * self.nq * (self.nq + 1) / 2)
+        import numpy as np
+        n16 = self.n // 16
+        words = self.union.cpu().numpy().view(np.uint32).reshape(-1, n16, self.union.shape[-1])
+        bits = np.unpackbits(words.view(np.uint8), axis=-1, bitorder="little")[..., :n16]
+        return float(np.tril(bits.astype(bool)).sum()) / (self.b * self.h * n16 * (n16 + 1) / 2)

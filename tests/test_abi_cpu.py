@@ -132,6 +132,26 @@ def test_control_and_support_mass_checks(lib):
     assert L.wise_support_mass(a, b, a + 64, lib.WiseShape(1, 2, 256, 80, 0.0, 0), None) == \
         lib.WISE_ERR_SHAPE
 
+
+def test_block16_checks(lib):
+    L = lib.lib
+    s = shape(lib)
+    a = 1 << 20
+    assert L.wise_block_mass_b16(None, a, a, a, s, None) == lib.WISE_ERR_ARG
+    assert L.wise_block_mass_b16(a, a, None, a, s, None) == lib.WISE_ERR_ARG
+    assert L.wise_block_mass_b16(a + 8, a, a, a, s, None) == lib.WISE_ERR_ALIGN
+    assert L.wise_select_union_b16(None, a, None, 0.95, s, None) == lib.WISE_ERR_ARG
+    assert L.wise_select_union_b16(a, a, None, 0.0, s, None) == lib.WISE_ERR_ARG
+    ws = L.wise_schedule_b16_workspace_bytes(s)
+    assert ws > L.wise_schedule_workspace_bytes(s)      # plus the folded 32-token masks
+    assert L.wise_build_schedule_b16(a, a, a, None, 10, None, a, ws, s, None) == lib.WISE_ERR_ARG
+    assert L.wise_build_schedule_b16(a, a, a, a, 10, None, a, ws - 1, s, None) == \
+        lib.WISE_ERR_WORKSPACE
+    assert L.wise_build_schedule_b16(a, a, a, a, 1, None, a, ws, s, None) == lib.WISE_ERR_CAPACITY
+    assert L.wise_sparse_attn_b16(a, a, a, a, a, a, None, 1, None, s, None) == lib.WISE_ERR_ARG
+    assert L.wise_sparse_attn_b16(a, a, a, a, a, a, a, -1, None, s, None) == lib.WISE_ERR_ARG
+    assert L.wise_sparse_attn_b16(a, a, a + 4, a, a, a, a, 1, None, s, None) == lib.WISE_ERR_ALIGN
+
 def test_schedule_sizes_and_checks(lib):
     L = lib.lib
     s = shape(lib, 1, 32, 4096, 128)

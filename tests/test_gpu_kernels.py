@@ -566,3 +566,141 @@ def test_bounded_wait_times_out_and_context_survives(ops):
     o, _, _ = ops.full_attn_mass(to_dev(qb), to_dev(kb), to_dev(vb))
     o_ref, _ = O.causal_attention(*(bf16_bits_to_f64(x[0, 0]) for x in (qb, kb, vb)))
     compare_o(dev_f32(o)[0, 0], o_ref)
+
+
+# ---------------------------------------------------------------- block size 16
+
+def _words_of(sel):
+    """[..., rows, cols] bool -> [..., rows, ceil(cols/32)] int32 words (bit c % 32 of word c // 32)."""
+    cols = sel.shape[-1]
+    W = (cols + 31) // 32
+    words = np.zeros(sel.shape[:-1] + (W,), np.uint32)
+    for c in range(cols):
+        words[..., c // 32] |= sel[..., c].astype(np.uint32) << np.uint32(c % 32)
+    return words.view(np.int32)
+
+
+def _decode_b16(ro, ci, sub, nq):
+    """One head's 32-token CSR plus sub-masks -> the 16-token support [2nq, 2nq]."""
+    sel = np.zeros((2 * nq, 2 * nq), bool)
+    for q in range(nq):
+        for e in range(ro[q], ro[q + 1]):
+            b = int(ci[e])
+            assert 0 < sub[e] < 16, "entries carry at least one sub-block"
+            for a in range(2):
+                for c in range(2):
+                    if (sub[e] >> (2 * a + c)) & 1:
+                        sel[2 * q + a, 2 * b + c] = True
+    return sel
+
+
+B16_SHAPES = [(1, 2, 256, 64), (2, 3, 544, 96), (1, 2, 1024, 128)]
+
+
+@pytest.mark.parametrize("b,h,n,d", B16_SHAPES)
+def test_block_mass_b16_matches_oracle(ops, b, h, n, d):
+    qb, kb, vb = rand_qkv_bits(b, h, n, d, seed=7 * n + d)
+    q, k, v = to_dev(qb), to_dev(kb), to_dev(vb)
+    _, lse, _ = ops.full_attn_mass(q, k, v, with_mass=False, lse=torch.empty(b, h, n, device="cuda"))
+    m16 = ops.block_mass_b16(q, k, lse).cpu().numpy()
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    n16 = n // 16
+    for bi in range(b):
+        for hi in range(h):
+            qf, kf = (bf16_bits_to_f64(x[bi, hi]) for x in (qb, kb))
+            r16 = O.block_mass(qf, kf, block=16)
+            assert np.abs(np.tril(m16[bi, hi]) - r16).max() <= MASS_TOL
+            # the one above-diagonal 16-block inside each diagonal 32-block is written 0
+            assert np.all(m16[bi, hi][np.arange(0, n16, 2), np.arange(1, n16, 2)] == 0.0)
+
+
+@pytest.mark.parametrize("n16,bh", [(16, 2), (90, 3), (1024, 1)])
+def test_select_union_b16_matches_oracle(ops, n16, bh):
+    rng = np.random.default_rng(n16 + 1)
+    m32 = _peaky_masses(rng, bh, n16).astype(np.float32)
+    union = ops.new_bitmask_b16(1, bh, n16 * 16, "cuda")
+    step = torch.empty_like(union)
+    ops.select_union_b16(torch.from_numpy(m32).reshape(1, bh, n16, n16).cuda(), union, 0.95,
+                         step_bits=step)
+    s = bits_to_bool(step.cpu().numpy()[0], n16)
+    assert np.array_equal(bits_to_bool(union.cpu().numpy()[0], n16), s)
+    exempt = sum(compare_selection(s[x], m32[x].astype(np.float64), 0.95) for x in range(bh))
+    assert exempt <= 2
+
+
+@pytest.mark.parametrize("nq,bh", [(1, 1), (5, 2), (45, 3), (512, 1)])
+def test_build_schedule_b16_bit_exact(ops, nq, bh):
+    """The schedule decodes back to exactly the causal part of the 16-token working set;
+    its 32-token CSR lists exactly the blocks with a kept sub-block, ascending."""
+    rng = np.random.default_rng(nq * 3 + bh)
+    n16 = 2 * nq
+    sel = rng.random((bh, n16, n16)) < 0.3           # includes bits above the diagonal
+    words = torch.from_numpy(_words_of(sel)).reshape(1, bh, n16, -1).cuda()
+    ro, ci, sub, nnz = ops.build_schedule_b16(words, head_dim=64)
+    ro, ci, sub = ro.cpu().numpy(), ci.cpu().numpy(), sub.cpu().numpy()
+    assert nnz == ro[-1]
+    for x in range(bh):
+        r0, r1 = x * nq, (x + 1) * nq
+        hro = ro[r0:r1 + 1] - ro[r0]
+        hci, hsub = ci[ro[r0]:ro[r1]], sub[ro[r0]:ro[r1]]
+        causal = np.tril(sel[x])
+        assert np.array_equal(_decode_b16(hro, hci, hsub, nq), causal)
+        fold = causal.reshape(nq, 2, nq, 2).any(axis=(1, 3))
+        check_csr(hro, hci, fold)
+
+
+def _b16_support(nq, rng, p=0.45, empty_row16=None):
+    sel = np.tril(rng.random((2 * nq, 2 * nq)) < p)
+    np.fill_diagonal(sel, True)
+    if empty_row16 is not None:
+        sel[empty_row16] = False
+    return sel
+
+
+@pytest.mark.parametrize("b,h,n,d,hkv", [(1, 2, 256, 64, 2), (1, 3, 544, 96, 3),
+                                         (2, 2, 1024, 128, 2), (1, 4, 512, 128, 1)])
+def test_sparse_attn_b16_matches_oracle(ops, b, h, n, d, hkv):
+    """Random 16-token supports (one 16-row left empty: O = 0, lse = -inf) through the GPU
+    schedule builder and the sub-masked kernel, against masked attention at B = 16."""
+    nq = n // 32
+    rng = np.random.default_rng(n + h)
+    qb, _, _ = rand_qkv_bits(b, h, n, d, seed=n + 5)
+    _, kb, vb = rand_qkv_bits(b, hkv, n, d, seed=n + 6)
+    sups = np.stack([_b16_support(nq, rng, empty_row16=(3 if x == 0 else None))
+                     for x in range(b * h)])
+    words = torch.from_numpy(_words_of(sups)).reshape(b, h, 2 * nq, -1).cuda()
+    ro, ci, sub, nnz = ops.build_schedule_b16(words, head_dim=d)
+    q, k, v = to_dev(qb), to_dev(kb), to_dev(vb)
+    lse = torch.empty(b, h, n, device="cuda")
+    o, _ = ops.sparse_attn_b16(q, k, v, ro, ci, sub, nnz, lse=lse)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    o, lse = dev_f32(o), lse.cpu().numpy()
+    g = h // hkv
+    for bi in range(b):
+        for hi in range(h):
+            x = bi * h + hi
+            qf = bf16_bits_to_f64(qb[bi, hi])
+            kf, vf = (bf16_bits_to_f64(t[bi, hi // g]) for t in (kb, vb))
+            o_ref, lse_ref = O.masked_attention(qf, kf, vf, sups[x], block=16)
+            rows = np.isfinite(lse_ref)
+            compare_o(o[bi, hi][rows], o_ref[rows], f"B16 O[{bi},{hi}]")
+            assert np.abs(lse[bi, hi][rows] - lse_ref[rows]).max() <= LSE_TOL
+            assert np.all(o[bi, hi][~rows] == 0.0) and np.all(np.isneginf(lse[bi, hi][~rows]))
+            if x == 0:
+                assert (~rows).sum() == 16
+
+
+def test_sparse_attn_b16_all_blocks_equals_dense(ops):
+    b, h, n, d = 1, 2, 544, 128
+    nq = n // 32
+    qb, kb, vb = rand_qkv_bits(b, h, n, d, seed=99)
+    q, k, v = to_dev(qb), to_dev(kb), to_dev(vb)
+    sel = np.broadcast_to(np.tril(np.ones((2 * nq, 2 * nq), bool)), (b * h, 2 * nq, 2 * nq))
+    words = torch.from_numpy(_words_of(np.ascontiguousarray(sel))).reshape(b, h, 2 * nq, -1).cuda()
+    ro, ci, sub, nnz = ops.build_schedule_b16(words, head_dim=d)
+    o16, _ = ops.sparse_attn_b16(q, k, v, ro, ci, sub, nnz)
+    od, _, _ = ops.full_attn_mass(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(o16, od)

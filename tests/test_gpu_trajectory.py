@@ -239,3 +239,60 @@ def test_trajectory_controls_and_retained_mass(support):
     assert exempt <= 3
     rfm = tr.retained_future_mass()
     assert 0.0 < rfm <= 1.0 + 1e-6
+
+
+# ------------------------------------------------------------- block size 16
+
+def test_trajectory_1k_block16():
+    """B = 16 (appendix C.6): window-step selections over 16-token masses against the
+    oracle's, the union, the schedule decoded back to the union, and late O against
+    masked attention at B = 16 over the GPU's union."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from recurrent_depth_lm_b200 import WiseTrajectory, ops
+    cfg = CONFIGS["1k"]
+    sample = [(0, 2), (0, 29)]
+    idx = [b * cfg.heads + h for (b, h) in sample]
+    nq, n16 = cfg.nq, cfg.seqlen // 16
+    check_steps = [13, 32]
+    tr = WiseTrajectory(cfg.batch, cfg.heads, cfg.seqlen, cfg.head_dim, t_d=cfg.t_d,
+                        window=cfg.window, eta=cfg.eta, block=16, keep_step_bits=True)
+    flat = lambda x: x.reshape(cfg.bh, *x.shape[2:])[idx]
+    o_late, bits = {}, {}
+    with StepPool(cfg, workers=max(1, min(16, os.cpu_count() or 2))) as pool:
+        for t, q, k, v in pool:
+            o = tr.step(t, _dev(q), _dev(k), _dev(v))
+            if tr.in_window(t):
+                bits[t] = bits_to_bool(flat(tr.step_bits[t]).cpu().numpy(), n16)
+            if t in check_steps:
+                o_late[t] = flat(o).float().cpu().numpy()
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    union = bits_to_bool(flat(tr.union).cpu().numpy(), n16)
+    ro_all, ci_all = tr.row_offsets.cpu().numpy(), tr.col_idx.cpu().numpy()
+    sub_all = tr.sub.cpu().numpy()
+    host = {t: (q, k, v) for t, q, k, v in iter_steps(cfg, heads=sample)}
+    exempt = 0
+    for si, bhi in enumerate(idx):
+        steps = []
+        for t in range(cfg.window[0], cfg.window[1] + 1):
+            q, k, _ = (bf16_bits_to_f64(x[si]) for x in host[t])
+            exempt += compare_selection(bits[t][si], O.block_mass(q, k, cfg.scale, block=16),
+                                        cfg.eta)
+            steps.append(bits[t][si])
+        assert np.array_equal(union[si], O.temporal_union(steps))
+        lo, hi = ro_all[bhi * nq], ro_all[(bhi + 1) * nq]
+        sel = np.zeros((n16, n16), bool)
+        for qq in range(nq):
+            for e in range(ro_all[bhi * nq + qq], ro_all[bhi * nq + qq + 1]):
+                for a in range(2):
+                    for c in range(2):
+                        if (sub_all[e] >> (2 * a + c)) & 1:
+                            sel[2 * qq + a, 2 * ci_all[e] + c] = True
+        assert hi >= lo and np.array_equal(sel, np.tril(union[si]))
+        for t in check_steps:
+            q, k, v = (bf16_bits_to_f64(x[si]) for x in host[t])
+            ref, _ = O.masked_attention(q, k, v, union[si], cfg.scale, block=16)
+            compare_o(o_late[t][si], ref, f"B16 head {sample[si]} step {t}")
+    assert exempt <= 2
+    assert 0.0 < tr.density() <= 1.0
