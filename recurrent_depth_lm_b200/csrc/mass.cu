@@ -6,8 +6,10 @@
 // every row i and admissible key block b the block's log2-sum-exp
 // blse_ib = log2 sum_{j in I_b, j <= i} 2^(s_ij * scale * log2 e); with the row's
 // final normaliser lse_i the inner sum is 2^(blse_ib - lse_i * log2 e).  This
-// kernel does the outer mean: one warp per (bh, q), lane = row of the query
-// block, a butterfly sum per key block.
+// kernel does the outer mean: one warp per (bh, q); lane l takes key blocks l,
+// l + 32, ... of the row and reads that block's 32 consecutive row values (blse is
+// [bh][key block][row]) as eight 16-byte loads, then sums them on its own, so a
+// warp keeps 4 KB of loads in flight and writes 128 consecutive bytes of mass.
 
 #include <cstdint>
 
@@ -24,30 +26,25 @@ __global__ void __launch_bounds__(256)
   if (row >= rows) return;  // warp-uniform
   const long long bh = row / nq;
   const int q = (int)(row % nq);
-  const int i = q * 32 + lane;
-  const float l2 = lse[bh * n + i] * 1.4426950408889634f;
-  const float* src = blse + bh * (long long)nq * n + i;
+  // log2-domain lse of the 32 rows of block q, every lane holding all 32
+  const float mine = lse[bh * n + q * 32 + lane] * 1.4426950408889634f;
+  float l2[32];
+#pragma unroll
+  for (int r = 0; r < 32; ++r) l2[r] = __shfl_sync(0xffffffffu, mine, r);
+  const float* base = blse + bh * (long long)nq * n + q * 32;
   float* dst = mass + (bh * nq + q) * (long long)nq;
-  // four key blocks per round: independent butterflies
-  for (int b0 = 0; b0 <= q; b0 += 4) {
-    float v[4];
+  for (int b = lane; b <= q; b += 32) {
+    const float4* src = reinterpret_cast<const float4*>(base + (long long)b * n);
+    float4 x[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int b = b0 + u;
-      v[u] = b <= q ? fast_exp2(src[(long long)b * n] - l2) : 0.f;
+    for (int u = 0; u < 8; ++u) x[u] = __ldg(src + u);
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      a0 += fast_exp2(x[u].x - l2[4 * u]) + fast_exp2(x[u].y - l2[4 * u + 1]);
+      a1 += fast_exp2(x[u].z - l2[4 * u + 2]) + fast_exp2(x[u].w - l2[4 * u + 3]);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] += __shfl_xor_sync(0xffffffffu, v[u], o);
-    }
-    if (lane < 4 && b0 + lane <= q) {
-      float mine = v[0];
-#pragma unroll
-      for (int u = 1; u < 4; ++u)
-        if (lane == u) mine = v[u];
-      dst[b0 + lane] = mine * (1.0f / 32.0f);
-    }
+    dst[b] = (a0 + a1) * (1.0f / 32.0f);
   }
 }
 
