@@ -836,52 +836,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           continue;
         }
 
-        // -------- pass 1: row max over the visible key blocks (log2 domain), two blocks
-        // per TMEM round trip
-        float mx;
-        {
-          float mxa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-          for (int s0 = 0; s0 < kSlots; s0 += 2) {
-            uint32_t sr[2][32];
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-              if ((vmask >> (s0 + h)) & 1u) tmem_ld32(t_lane + s_col + (s0 + h) * 32, sr[h]);
-            tmem_wait_ld();
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              if (!((vmask >> (s0 + h)) & 1u)) continue;
-              reg_fence(sr[h]);
-              if ((dmask >> (s0 + h)) & 1u) {
-#pragma unroll
-                for (int c = 0; c < 32; ++c)
-                  if (c > lane) sr[h][c] = __float_as_uint(-INFINITY);
-              }
-              if (MODE == kModeSparse16 && ((hmask >> (2 * (s0 + h))) & 3u) != 3u)
-                half_mask(sr[h], (hmask >> (2 * (s0 + h))) & 3u);
-#pragma unroll
-              for (int c = 0; c < 32; c += 8) {
-#pragma unroll
-                for (int y = 0; y < 4; ++y)
-                  mxa[y] = max3(mxa[y], __uint_as_float(sr[h][c + 2 * y]),
-                                __uint_as_float(sr[h][c + 2 * y + 1]));
-              }
-            }
-          }
-          mx = max3(mxa[0], mxa[1], fmaxf(mxa[2], mxa[3])) * sl2;
-        }
-        const float m_new = fmaxf(m, mx);
-        const bool need = m_new > m + 8.0f;   // true on the first finite score
-        const bool warp_need = __any_sync(0xffffffffu, need);
-        const float m_use = warp_need ? m_new : m;
-        const float alpha = (warp_need && m != -INFINITY) ? fast_exp2(m - m_use) : 1.0f;
-        const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;  // all scores are -inf then
-        const uint64_t sc2 = f2(sl2, sl2), nm2 = f2(neg_m, neg_m);
-
-        // -------- pass 2: P = 2^(s*scale*log2e - m) as bf16 pairs over S_X columns [0, 64)
-        // Key block s goes to P columns [16 s, 16 s + 16), which lie in S columns of
-        // blocks <= s that this pass has already read.
+        // -------- one pass over the entry's key blocks: P = 2^(s*scale*log2e - m_ref) as
+        // bf16 pairs over S_X columns [0, 64).  Key block s goes to P columns
+        // [16 s, 16 s + 16), which lie below S block s: reading S block s never sees P.
+        // m_ref is the row's exponent reference; it moves only when a block's max
+        // exceeds it by more than 2^8, and then the P blocks already written (and the
+        // row sum) are rescaled in place, so every P of the entry shares one reference.
+        float m_ref = m;
         float rs = 0.f;
+        const uint64_t sc2 = f2(sl2, sl2);
+        auto rescale_p = [&](int s, float f) {
+          tmem_wait_st();   // the P stores of the earlier blocks have landed
+#pragma unroll 1
+          for (int t = 0; t < s; ++t) {
+            if (!((vmask >> t) & 1u)) continue;   // P = 0 there
+            uint32_t w[16];
+            tmem_ld16(t_lane + s_col + t * 16, w);
+            tmem_wait_ld();
+            reg_fence(w);
+#pragma unroll
+            for (int y = 0; y < 16; ++y) {
+              const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&w[y]);
+              w[y] = pack_bf16x2(__low2float(h) * f, __high2float(h) * f);
+            }
+            tmem_st16(t_lane + s_col + t * 16, w);
+          }
+        };
         auto block_exp = [&](uint32_t (&v)[32], int s) {
           uint32_t w[16];
           if ((vmask >> s) & 1u) {
@@ -893,6 +873,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (MODE == kModeSparse16 && ((hmask >> (2 * s)) & 3u) != 3u)
               half_mask(v, (hmask >> (2 * s)) & 3u);
+            float mxa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < 32; c += 8) {
+#pragma unroll
+              for (int y = 0; y < 4; ++y)
+                mxa[y] = max3(mxa[y], __uint_as_float(v[c + 2 * y]), __uint_as_float(v[c + 2 * y + 1]));
+            }
+            const float bm = max3(mxa[0], mxa[1], fmaxf(mxa[2], mxa[3])) * sl2;
+            const bool trig = bm > m_ref + 8.0f;   // true on the row's first finite score
+            if (__any_sync(0xffffffffu, trig)) {
+              const float m_new = trig ? bm : m_ref;
+              const float f = trig ? fast_exp2(m_ref - m_new) : 1.0f;   // 0 from -inf
+              rescale_p(s, f);
+              rs *= f;
+              m_ref = m_new;
+            }
+            const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;  // all scores -inf then
+            const uint64_t nm2 = f2(neg_m, neg_m);
             uint64_t rs2[2] = {0ull, 0ull};
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
@@ -912,7 +910,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               // into block mass with the final lse.  Layout [bh][key block][row]: 32
               // lanes store 32 consecutive floats.
               p.blse[((long long)bh * p.nq + e.kb[s]) * p.n + i] =
-                  ps > 0.f ? m_use + __log2f(ps) : -INFINITY;
+                  ps > 0.f ? m_ref + __log2f(ps) : -INFINITY;
             }
           } else {
 #pragma unroll
@@ -929,6 +927,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           block_exp(v, s);
         }
+        const bool need = m_ref != m;   // this row's reference moved during the entry
+        const bool warp_need = __any_sync(0xffffffffu, need);
+        const float alpha = (need && m != -INFINITY) ? fast_exp2(m - m_ref) : 1.0f;
+        const float m_use = m_ref;
         if (warp_need && !first) {
           // O_X is rescaled in place.  Its last PV has completed: QK_X of this entry
           // was issued only after it.

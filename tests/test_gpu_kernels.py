@@ -4,6 +4,8 @@ Sizes span several 128-row tiles, ragged tails (seqlen not a multiple of 128,
 a single 32-token block), every supported head_dim and batch*heads > 1.
 """
 
+import math
+
 import numpy as np
 import pytest
 
@@ -704,3 +706,42 @@ def test_sparse_attn_b16_all_blocks_equals_dense(ops):
     od, _, _ = ops.full_attn_mass(q, k, v)
     torch.cuda.synchronize()
     assert torch.equal(o16, od)
+
+
+# ---------------------------------------------------------------- score jumps inside an entry
+
+@pytest.mark.parametrize("jump", [20.0, 200.0])
+def test_score_jump_inside_an_entry(ops, jump):
+    """Key block 3 scores `jump` (log2 units) above blocks 0-2 for every query that sees
+    it: the softmax meets a row max far above its running reference partway through an
+    entry of 4 key blocks, after P of the earlier blocks is written (and, at 200, beyond
+    the fp32 range of 2^-126 for those earlier blocks).  Dense and all-blocks sparse
+    against the oracle."""
+    b, h, n, d = 1, 2, 256, 64
+    rng = np.random.default_rng(int(jump))
+    q = rng.standard_normal((b, h, n, d), dtype=np.float32) * np.float32(0.3)
+    k = rng.standard_normal((b, h, n, d), dtype=np.float32) * np.float32(0.3)
+    v = rng.standard_normal((b, h, n, d), dtype=np.float32)
+    scale = 1.0 / math.sqrt(d)
+    q[..., 0] = 1.0
+    k[..., 0] = 0.0
+    k[:, :, 96:128, 0] = np.float32(jump / (scale * math.log2(math.e)))
+    qb, kb, vb = (f32_to_bf16_bits(x) for x in (q, k, v))
+    dq, dk, dv = to_dev(qb), to_dev(kb), to_dev(vb)
+    nq = n // 32
+    per_head = nq * (nq + 1) // 2
+    ro = torch.tensor([x * per_head + r * (r + 1) // 2 for x in range(b * h) for r in range(nq)]
+                      + [b * h * per_head], dtype=torch.int32, device="cuda")
+    ci = torch.tensor([c for x in range(b * h) for r in range(nq) for c in range(r + 1)],
+                      dtype=torch.int32, device="cuda")
+    od, lse_d, _ = ops.full_attn_mass(dq, dk, dv, lse=torch.empty(b, h, n, device="cuda"))
+    lse_s = torch.empty(b, h, n, device="cuda")
+    os_, _ = ops.sparse_attn(dq, dk, dv, ro, ci, ci.numel(), lse=lse_s)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    for hi in range(h):
+        qf, kf, vf = (bf16_bits_to_f64(x[0, hi]) for x in (qb, kb, vb))
+        o_ref, lse_ref = O.causal_attention(qf, kf, vf)
+        for name, o, l in (("dense", od, lse_d), ("sparse", os_, lse_s)):
+            compare_o(dev_f32(o)[0, hi], o_ref, f"{name} jump {jump} head {hi}")
+            assert np.abs(l.cpu().numpy()[0, hi] - lse_ref).max() <= LSE_TOL
