@@ -1,0 +1,95 @@
+"""Host-side logic that needs no GPU: trajectory argument checks, the 16-token density
+count, bench.py's workload overrides and FLOP accounting."""
+
+import argparse
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def traj_cls():
+    from recurrent_depth_lm_b200.trajectory import WiseTrajectory
+    return WiseTrajectory
+
+
+def make(traj_cls, **kw):
+    args = dict(batch=1, heads=2, seqlen=256, head_dim=64, device="cpu")
+    args.update(kw)
+    return traj_cls(args.pop("batch"), args.pop("heads"), args.pop("seqlen"),
+                    args.pop("head_dim"), **args)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(block=48),                                   # not a supported block size
+    dict(block=128, seqlen=192),                      # seqlen not a multiple of the block
+    dict(support="oracle"),                           # unknown support
+    dict(support="size_matched", block=64),           # controls are defined at B = 32
+    dict(support="mass_matched", block=16),
+    dict(support="static95", block=16),               # B = 16 runs the WISE support only
+    dict(block=16, track_retained=True),
+])
+def test_trajectory_rejects_bad_arguments(traj_cls, kw):
+    with pytest.raises(ValueError):
+        make(traj_cls, **kw)
+
+
+def test_late_step_before_schedule_and_untracked_retained_mass(traj_cls):
+    tr = make(traj_cls)
+    x = torch.zeros(1, 2, 256, 64, dtype=torch.bfloat16)
+    with pytest.raises(RuntimeError):
+        tr.step(tr.t_d + 1, x, x, x)
+    with pytest.raises(RuntimeError):
+        tr.retained_future_mass()
+
+
+def test_block16_density_counts_causal_16_token_blocks(traj_cls):
+    tr = make(traj_cls, block=16, seqlen=320)
+    n16 = 320 // 16
+    rng = np.random.default_rng(0)
+    sel = rng.random((2, n16, n16)) < 0.4
+    words = np.zeros((2, n16, tr.union.shape[-1]), np.uint32)
+    for b in range(n16):
+        words[..., b // 32] |= sel[..., b].astype(np.uint32) << np.uint32(b % 32)
+    tr.union.copy_(torch.from_numpy(words.view(np.int32)).reshape(tr.union.shape))
+    want = np.tril(sel).sum() / (2 * n16 * (n16 + 1) / 2)
+    assert abs(tr.density() - want) < 1e-12
+
+
+def _args(**kw):
+    base = dict(config="4k", eta=None, t_d=None, window=None)
+    base.update(kw)
+    return argparse.Namespace(**base)
+
+
+def test_bench_workload_overrides():
+    import bench
+    cfg = bench.workload(_args())
+    assert (cfg.eta, cfg.t_d, cfg.window) == (0.95, 12, (9, 12))
+    cfg = bench.workload(_args(eta=0.9, t_d=8))
+    assert (cfg.eta, cfg.t_d, cfg.window) == (0.9, 8, (5, 8))     # window follows t_d
+    cfg = bench.workload(_args(window=[11, 12]))
+    assert cfg.window == (11, 12) and cfg.t_d == 12
+    with pytest.raises(SystemExit):
+        bench.workload(_args(window=[10, 14]))                      # past t_d
+    with pytest.raises(SystemExit):
+        bench.workload(_args(t_d=32))                               # no late step left
+
+
+def test_bench_flops_b16_counts_pairs_inside_kept_blocks():
+    """4*d per admissible pair: 16*16 per kept off-diagonal 16-block, 16*17/2 per diagonal."""
+    import bench
+    from wise_inputs import CONFIGS
+    cfg = CONFIGS["tiny"]                             # n = 256: 16 blocks of 16 tokens
+    n16 = cfg.seqlen // 16
+    sel = np.zeros((cfg.bh, n16, n16), bool)
+    sel[0, 5, 5] = True                               # diagonal
+    sel[0, 5, 2] = True                               # off-diagonal
+    sel[1, 3, 7] = True                               # above the diagonal: not counted
+    words = np.zeros((cfg.bh, n16, 1), np.uint32)
+    for b in range(n16):
+        words[..., 0] |= sel[..., b].astype(np.uint32) << np.uint32(b)
+    flops = bench.sparse_flops_b16(cfg, words.view(np.int32))
+    assert flops == 4.0 * cfg.head_dim * (256 + 136)
