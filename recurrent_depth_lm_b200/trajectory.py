@@ -177,6 +177,49 @@ class WiseTrajectory:
             raise RuntimeError("no late step ran with track_retained=True")
         return float(torch.stack(list(self.retained.values())).mean().item())
 
+    # ------------------------------------------------------------ save / replay
+    def state(self) -> dict:
+        """The frozen working set and its schedule as host arrays.  Late steps depend on
+        nothing else, so a loaded state replays them without the exploration steps."""
+        import numpy as np
+        if not self.scheduled:
+            raise RuntimeError("no schedule yet: run the steps up to t_d first")
+        nnz = self.nnz()
+        st = {
+            "shape": np.array([self.b, self.h, self.n, self.d, self.block], np.int64),
+            "t_d": np.array(self.t_d), "window": np.array(self.window), "eta": np.array(self.eta),
+            "support": np.array(self.support),
+            "frozen": self.frozen.cpu().numpy(),
+            "row_offsets": self.row_offsets.cpu().numpy(),
+            "col_idx": self.col_idx[:nnz].cpu().numpy(),
+        }
+        if self.sub is not None:
+            st["sub"] = self.sub[:nnz].cpu().numpy()
+        return st
+
+    def save(self, path) -> None:
+        import numpy as np
+        np.savez(path, **self.state())
+
+    def load(self, path_or_state) -> None:
+        """Restore a saved working set and schedule; the next step may be any t > t_d."""
+        import numpy as np
+        st = path_or_state if isinstance(path_or_state, dict) else dict(np.load(path_or_state))
+        want = np.array([self.b, self.h, self.n, self.d, self.block], np.int64)
+        if not np.array_equal(np.asarray(st["shape"]), want):
+            raise ValueError(f"saved shape/block {st['shape'].tolist()} != {want.tolist()}")
+        col = np.asarray(st["col_idx"], np.int32)
+        ro = np.asarray(st["row_offsets"], np.int32)
+        if ro.shape != tuple(self.row_offsets.shape) or col.size > self.col_idx.numel() or \
+                (ro.size and int(ro[-1]) != col.size):
+            raise ValueError("saved schedule does not fit this trajectory")
+        self.frozen.copy_(torch.from_numpy(np.asarray(st["frozen"], np.int32)))
+        self.row_offsets.copy_(torch.from_numpy(ro))
+        self.col_idx[:col.size].copy_(torch.from_numpy(col))
+        if self.sub is not None:
+            self.sub[:col.size].copy_(torch.from_numpy(np.asarray(st["sub"], np.uint8)))
+        self.scheduled = True
+
     def nnz(self) -> int:
         return int(self.row_offsets[-1].item())
 

@@ -296,3 +296,29 @@ def test_trajectory_1k_block16():
             compare_o(o_late[t][si], ref, f"B16 head {sample[si]} step {t}")
     assert exempt <= 2
     assert 0.0 < tr.density() <= 1.0
+
+
+def test_saved_working_set_replays_late_steps(tmp_path):
+    """A trajectory restored from a saved working set runs the late steps alone and gives
+    bit-identical outputs (the schedule is all the late steps depend on)."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from recurrent_depth_lm_b200 import WiseTrajectory
+    cfg = CONFIGS["tiny"]
+    mk = lambda: WiseTrajectory(cfg.batch, cfg.heads, cfg.seqlen, cfg.head_dim, t_d=cfg.t_d,
+                                window=cfg.window, eta=cfg.eta)
+    tr = mk()
+    late = {}
+    with StepPool(cfg, workers=2) as pool:
+        for t, q, k, v in pool:
+            x = (_dev(q), _dev(k), _dev(v))
+            o = tr.step(t, *x)
+            if t > cfg.t_d:
+                late[t] = (x, o.clone())
+    path = tmp_path / "working_set.npz"
+    tr.save(path)
+    tr2 = mk()
+    tr2.load(path)
+    for t, (x, o) in late.items():
+        assert torch.equal(tr2.step(t, *x), o)
+    torch.cuda.synchronize()

@@ -93,3 +93,43 @@ def test_bench_flops_b16_counts_pairs_inside_kept_blocks():
         words[..., 0] |= sel[..., b].astype(np.uint32) << np.uint32(b)
     flops = bench.sparse_flops_b16(cfg, words.view(np.int32))
     assert flops == 4.0 * cfg.head_dim * (256 + 136)
+
+
+def _fake_schedule(tr, rng):
+    """A random causal working set and its CSR written into a CPU trajectory's buffers."""
+    from oracle import wise_oracle as O
+    nq = tr.nq
+    words = np.zeros(tuple(tr.union.shape), np.uint32)
+    ro_all, ci_all = [0], []
+    for x in range(tr.b * tr.h):
+        sup = np.tril(rng.random((nq, nq)) < 0.5)
+        np.fill_diagonal(sup, True)
+        for b in range(nq):
+            words[0, x, :, b // 32] |= sup[:, b].astype(np.uint32) << np.uint32(b % 32)
+        ro, ci = O.csr_schedule(sup)
+        ro_all += (ro[1:] + ro_all[-1]).tolist()
+        ci_all += ci.tolist()
+    tr.union.copy_(torch.from_numpy(words.view(np.int32)))
+    tr.row_offsets.copy_(torch.tensor(ro_all, dtype=torch.int32))
+    tr.col_idx[:len(ci_all)].copy_(torch.tensor(ci_all, dtype=torch.int32))
+    tr.scheduled = True
+    return len(ci_all)
+
+
+def test_save_and_load_round_trip(traj_cls, tmp_path):
+    tr = make(traj_cls, heads=3, seqlen=320)
+    with pytest.raises(RuntimeError):
+        tr.state()                                     # nothing frozen yet
+    nnz = _fake_schedule(tr, np.random.default_rng(5))
+    path = tmp_path / "ws.npz"
+    tr.save(path)
+    tr2 = make(traj_cls, heads=3, seqlen=320)
+    tr2.load(path)
+    assert tr2.scheduled and tr2.nnz() == nnz
+    assert torch.equal(tr2.union, tr.union)
+    assert torch.equal(tr2.row_offsets, tr.row_offsets)
+    assert torch.equal(tr2.col_idx[:nnz], tr.col_idx[:nnz])
+    with pytest.raises(ValueError):
+        make(traj_cls, heads=3, seqlen=256).load(path)     # another shape
+    with pytest.raises(ValueError):
+        make(traj_cls, heads=3, seqlen=320, block=64).load(path)   # another block size
