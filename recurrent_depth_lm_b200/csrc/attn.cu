@@ -1,9 +1,12 @@
 // attn.cu -- tcgen05/TMEM attention kernels of the WISE hot path (sm_100a).
 //
-// One persistent, warp-specialised kernel template covers three modes:
-//   kDense  : exploration-step causal attention (all admissible key blocks),
-//   kSparse : late-step attention over a CSR key-block schedule,
-//   kMass   : the block-mass pass of an exploration window step (two-pass path).
+// One persistent, warp-specialised kernel template covers four modes:
+//   kDense    : exploration-step causal attention (all admissible key blocks), which
+//               can also record per-(row, key block) log-sum-exps for the block mass,
+//   kSparse   : late-step attention over a CSR key-block schedule,
+//   kMass     : the block-mass pass with Q K^T recomputed (two-pass path; also the
+//               16-token block mass),
+//   kSparse16 : kSparse whose entries carry 16 x 16 sub-block masks (block size 16).
 //
 // Semantics follow Wan & Chen, "Attention Routing Stabilizes Early:
 // Working-Set Inference for Recurrent-Depth Language Models": section 3
@@ -39,6 +42,8 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+
+#include <atomic>
 #include <cstdint>
 
 #include "sm100.cuh"
@@ -715,9 +720,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   } else {
     // ======================================================= softmax / epilogue of slot X
-    // Thread = row.  Each iteration reads its key blocks from S_X twice (row max,
-    // then exponentials), one 32-column block at a time in a rolled loop: the hot
-    // loop stays small enough for the instruction cache.
+    // Thread = row.  Each iteration reads its key blocks from S_X once, one 32-column
+    // block at a time in a rolled loop (block max, then exponentials against the row's
+    // reference): the hot loop stays small enough for the instruction cache.
     const int X = (warp - 4) >> 2;
     const int qw = warp & 3;            // TMEM lane quarter = query block within the tile
     const uint32_t t_lane = tmem_base + ((uint32_t)(qw * 32) << 16);
@@ -1000,12 +1005,19 @@ static cudaError_t launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, con
                                const AttnParams& p, int grid, cudaStream_t stream,
                                const char** why) {
   using C = Cfg<D, MODE>;
-  static bool configured = false;  // per instantiation; attribute is per function
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, MODE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  // The shared-memory limit is a per-device attribute of the function: set it once per
+  // device (a repeated set from racing threads is harmless).
+  constexpr int kDevs = 64;
+  static std::atomic<bool> configured[kDevs];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kDevs) return cudaErrorInvalidDevice;
+  if (!configured[dev].load(std::memory_order_acquire)) {
+    e = cudaFuncSetAttribute(attn_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    configured = true;
+    configured[dev].store(true, std::memory_order_release);
   }
   attn_kernel<D, MODE><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
