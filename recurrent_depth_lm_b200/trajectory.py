@@ -55,15 +55,17 @@ class WiseTrajectory:
         self.scale = scale
         dev = torch.device(device)
         self.lse = torch.empty(batch, heads, seqlen, dtype=torch.float32, device=dev)
-        self.mass = torch.empty(batch, heads, self.nq, self.nq, dtype=torch.float32, device=dev)
-        self.union = ops.new_bitmask(batch, heads, self.nq, dev)
-        self.mass16 = self.sub = self.ws16 = None
+        self.mass16 = self.sub = self.mass = self.mass_ws = None
         if block == 16:   # 16-token masses and working set; sub-masks of the schedule
             self.mass16 = torch.empty(batch, heads, seqlen // 16, seqlen // 16,
                                       dtype=torch.float32, device=dev)
             self.union = ops.new_bitmask_b16(batch, heads, seqlen, dev)
-        # per-(row, key block) log-sum-exps of the one-pass block mass (window steps)
-        self.mass_ws = ops.mass_workspace(batch, heads, seqlen, head_dim, dev)
+        else:
+            self.mass = torch.empty(batch, heads, self.nq, self.nq, dtype=torch.float32,
+                                    device=dev)
+            self.union = ops.new_bitmask(batch, heads, self.nq, dev)
+            # per-(row, key block) log-sum-exps of the one-pass block mass (window steps)
+            self.mass_ws = ops.mass_workspace(batch, heads, seqlen, head_dim, dev)
         self.step_bits = {}
         self.keep_step_bits = keep_step_bits
         self.row_offsets = torch.empty(batch * heads * self.nq + 1, dtype=torch.int32, device=dev)
