@@ -370,6 +370,18 @@ def test_union_and_csr_invariants():
     assert np.array_equal(O.support_from_csr(ro, ci, nq), U)
 
 
+
+def test_block_density_exact_values():
+    """Fraction of the nq(nq+1)/2 causal blocks kept: all causal -> 1, diagonal only ->
+    2/(nq+1), blocks above the diagonal never count."""
+    nq = 9
+    assert O.block_density(np.tril(np.ones((nq, nq), bool))) == 1.0
+    assert O.block_density(np.eye(nq, dtype=bool)) == 2.0 / (nq + 1)
+    assert O.block_density(np.triu(np.ones((nq, nq), bool), 1)) == 0.0
+    sup = np.zeros((nq, nq), bool)
+    sup[4, :3] = True
+    assert O.block_density(sup | np.triu(np.ones((nq, nq), bool), 1)) == 3 / 45
+
 # --------------------------------------------------------------------------- sparse attention
 
 def test_all_blocks_schedule_equals_dense():
