@@ -181,3 +181,36 @@ def test_last_error_is_thread_local(lib):
     t.join()
     assert seen["msg"] == ""
     assert lib.last_error() != ""
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/wise.h compiles as C99 (no C++ or torch types), and a C program linked
+    against libwise.so calls it: version string, a shape error with its message."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    pkg = os.path.join(ROOT, "recurrent_depth_lm_b200")
+    src = tmp_path / "use_wise.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "wise.h"
+int main(void) {
+  wise_shape_t s;
+  memset(&s, 0, sizeof s);
+  s.batch = 1; s.heads = 2; s.seqlen = 100; s.head_dim = 64;   /* seqlen not a multiple of 32 */
+  int rc = wise_select_union((const float*)0x1000, (uint32_t*)0x1000, NULL, 0.95f, s, NULL);
+  printf("%s|%d|%s\n", wise_version(), rc, wise_last_error());
+  return rc == WISE_ERR_SHAPE ? 0 : 1;
+}
+''')
+    exe = tmp_path / "use_wise"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-L", pkg, "-lwise", "-Wl,-rpath," + pkg, "-o", str(exe)],
+                   check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out.stdout + out.stderr
+    version, rc, msg = out.stdout.strip().split("|")
+    assert version and int(rc) < 0 and "seqlen" in msg
