@@ -23,7 +23,15 @@ Readings of points the paper leaves open (also listed in the design notes):
 * if no prefix reaches eta (eta >= 1, or rounding), every admissible block is
   selected, which makes eta = 1 reproduce dense causal attention;
 * admissible key blocks of query block q are b <= q (causal mask M of §3);
-* block masses come from the full, unrestricted causal softmax of that step.
+* block masses come from the full, unrestricted causal softmax of that step;
+* a row with no kept admissible key (only possible for supports the method
+  itself never produces) has O = 0 and lse = -inf;
+* block sizes other than 32 (App. C.6): the block mass is the same definition
+  at that size; 64 / 128-token supports run as 32 x 32 subtiles clipped to the
+  causal part of the coarse diagonal block;
+* MassMatched (App. B, whose formula for the control itself did not survive):
+  the fewest step-1-ranked blocks whose step-1 mass reaches that of the WISE
+  working set, with correctly rounded sums; TopK ties go to the lower index.
 """
 
 from __future__ import annotations
