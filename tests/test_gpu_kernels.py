@@ -745,3 +745,23 @@ def test_score_jump_inside_an_entry(ops, jump):
         for name, o, l in (("dense", od, lse_d), ("sparse", os_, lse_s)):
             compare_o(dev_f32(o)[0, hi], o_ref, f"{name} jump {jump} head {hi}")
             assert np.abs(l.cpu().numpy()[0, hi] - lse_ref).max() <= LSE_TOL
+
+
+def test_sparse_attn_b16_maximum_length(ops):
+    """n = 16384 (512 query blocks: every word of the sub-mask planes in use), one head
+    against masked attention at B = 16."""
+    b, h, n, d = 1, 1, 16384, 64
+    nq = n // 32
+    rng = np.random.default_rng(16384)
+    qb, kb, vb = rand_qkv_bits(b, h, n, d, seed=77)
+    sel = _b16_support(nq, rng, p=0.3)
+    words = torch.from_numpy(_words_of(sel[None])).reshape(b, h, 2 * nq, -1).cuda()
+    ro, ci, sub, nnz = ops.build_schedule_b16(words, head_dim=d)
+    lse = torch.empty(b, h, n, device="cuda")
+    o, _ = ops.sparse_attn_b16(to_dev(qb), to_dev(kb), to_dev(vb), ro, ci, sub, nnz, lse=lse)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    qf, kf, vf = (bf16_bits_to_f64(x[0, 0]) for x in (qb, kb, vb))
+    o_ref, lse_ref = O.masked_attention(qf, kf, vf, sel, block=16)
+    compare_o(dev_f32(o)[0, 0], o_ref, "B16 n=16384")
+    assert np.abs(lse.cpu().numpy()[0, 0] - lse_ref).max() <= LSE_TOL
