@@ -58,3 +58,37 @@ def test_single_process_reductions_are_identity():
     import bench
     assert bench.reduce_max(3.5, torch.device("cpu")) == 3.5
     assert bench.reduce_sum(2.0, torch.device("cpu")) == 2.0
+
+
+def test_reference_arm_json_contract(capsys, monkeypatch):
+    """`bench.py --impl reference` prints one JSON line with the contract's keys (the
+    oracle timed on the host on a bounded sample); a non-zero rank prints nothing."""
+    import json
+
+    import bench
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    bench.main(["--impl", "reference", "--config", "tiny", "--steps", "1", "--warmup", "3",
+                "--eta", "0.9"])
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    assert "eta=0.9" in d["config"]["workload"]
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    bench.main(["--impl", "reference", "--config", "tiny", "--steps", "1", "--warmup", "3"])
+    assert capsys.readouterr().out.strip() == ""
+
+
+def test_bench_rejects_fewer_than_three_warmups():
+    import bench
+    with pytest.raises(SystemExit):
+        bench.main(["--impl", "reference", "--config", "tiny", "--steps", "1", "--warmup", "2"])
