@@ -543,6 +543,7 @@ def bench_wise(args):
                                + ({16: " (32x32 tiles with 16x16 sub-masks)", 32: ""}
                                   .get(args.block, " (run as 32x32 subtiles)")),
                    "step": "one full WISE trajectory (dense + mass/select + schedule + sparse)",
+                   "seed": f"[{cfg.seed}, rank, batch, head] per head (PCG64)",
                    "l2": "inputs larger than L2: every trajectory streams "
                          f"{3 * cfg.steps * cfg.bh * cfg.seqlen * cfg.head_dim * 2 / 1e9:.2f} GB "
                          "of fresh Q/K/V",
