@@ -668,14 +668,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!warp_wait(bar_q_full(X), S.qtiles & 1, abort_flag, p.status)) return false;
           ++S.qtiles;
         }
-        if (S.qkc >= 1) {
-          // S_X holds the previous P_X (read by the PV just issued) or, in mass mode, the
-          // previous S_X (read by the softmax warps)
-          const bool w = C::kAttn
-                             ? warp_wait(bar_o_done(X), (S.pvc - 1) & 1, abort_flag, p.status)
-                             : warp_wait(bar_s_free(X), (S.qkc - 1) & 1, abort_flag, p.status);
-          if (!w) return false;
-        }
+        // Attention modes: S_X holds P_X, which the PV just issued reads.  tcgen05 MMAs
+        // issued by one thread execute in issue order, so this QK overwrites S_X only
+        // after that PV has read it, with no wait for the PV here; and the s_full commit
+        // below tracks the PV too, so the softmax may rescale O_X once S_X is ready.
+        // Mass mode: the softmax warps read S_X itself, so wait until they are done.
+        if (!C::kAttn && S.qkc >= 1 &&
+            !warp_wait(bar_s_free(X), (S.qkc - 1) & 1, abort_flag, p.status))
+          return false;
         tc_fence_after();
         const uint32_t idesc = idesc_bf16_f32(128, 32 * ns, 0, 0);
         const uint32_t d_tmem = tmem_base + X * 128;
@@ -734,7 +734,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool run = true;
     while (run) {
       // ---------------- one tile of the slot: its entries, then the epilogue
-      float m = -INFINITY, l = 0.f, lse_l2 = 0.f;
+      float m = -INFINITY, l = 0.f, l32 = 0.f, lse_l2 = 0.f;
       int bh = 0, qb = 0, i = 0;
       bool first = true;
       while (true) {
@@ -844,11 +844,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // -------- one pass over the entry's key blocks: P = 2^(s*scale*log2e - m_ref) as
         // bf16 pairs over S_X columns [0, 64).  Key block s goes to P columns
         // [16 s, 16 s + 16), which lie below S block s: reading S block s never sees P.
-        // m_ref is the row's exponent reference; it moves only when a block's max
-        // exceeds it by more than 2^8, and then the P blocks already written (and the
-        // row sum) are rescaled in place, so every P of the entry shares one reference.
+        // m_ref is the row's exponent reference, an integer: it moves only when a block's
+        // max exceeds it by more than 2^8, and then the P blocks already written (and the
+        // row sums) are rescaled in place by an exact power of two, so every P of the
+        // entry shares one reference and no value is rounded twice.
+        // rs sums the fp32 P (it gives the log-sum-exps); rcorr adds, per key block, the
+        // bf16 rounding error of the block's largest P.  O is normalised by rs + rcorr: the
+        // PV MMA multiplies the bf16-rounded P into V, and where a few keys carry the
+        // row's weight the rounding of those P is what would otherwise bias O.
         float m_ref = m;
-        float rs = 0.f;
+        float rs = 0.f, rcorr = 0.f;
         const uint64_t sc2 = f2(sl2, sl2);
         auto rescale_p = [&](int s, float f) {
           tmem_wait_st();   // the P stores of the earlier blocks have landed
@@ -885,13 +890,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int y = 0; y < 4; ++y)
                 mxa[y] = max3(mxa[y], __uint_as_float(v[c + 2 * y]), __uint_as_float(v[c + 2 * y + 1]));
             }
-            const float bm = max3(mxa[0], mxa[1], fmaxf(mxa[2], mxa[3])) * sl2;
+            const float bmax = max3(mxa[0], mxa[1], fmaxf(mxa[2], mxa[3]));
+            const float bm = bmax * sl2;
             const bool trig = bm > m_ref + 8.0f;   // true on the row's first finite score
             if (__any_sync(0xffffffffu, trig)) {
-              const float m_new = trig ? bm : m_ref;
-              const float f = trig ? fast_exp2(m_ref - m_new) : 1.0f;   // 0 from -inf
+              const float m_new = trig ? ceilf(bm) : m_ref;
+              const float f = trig ? exp2_int(m_ref - m_new) : 1.0f;   // 0 from -inf
               rescale_p(s, f);
               rs *= f;
+              rcorr *= f;
               m_ref = m_new;
             }
             const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;  // all scores -inf then
@@ -909,6 +916,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             f2_split(add2(rs2[0], rs2[1]), lo, hi);
             const float ps = lo + hi;
             rs += ps;
+            {
+              // the block's largest P, computed as its element was, and its bf16 rounding
+              const float pm = fast_exp2(fmaf(bmax, sl2, neg_m));
+              rcorr += __uint_as_float(pack_bf16x2(pm, 0.f) << 16) - pm;
+            }
             if (MODE == kModeDense && p.blse != nullptr) {
               // block log-sum-exp of this row over key block kb, log2 domain:
               // blse = m + log2(sum_j 2^(s_ij*scale*log2e - m)); the mass pass turns it
@@ -934,7 +946,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const bool need = m_ref != m;   // this row's reference moved during the entry
         const bool warp_need = __any_sync(0xffffffffu, need);
-        const float alpha = (need && m != -INFINITY) ? fast_exp2(m - m_ref) : 1.0f;
+        const float alpha = (need && m != -INFINITY) ? exp2_int(m - m_ref) : 1.0f;
         const float m_use = m_ref;
         if (warp_need && !first) {
           // O_X is rescaled in place.  Its last PV has completed: QK_X of this entry
@@ -955,7 +967,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar_p_full(X));
         mbar_arrive(bar_e_empty(X, k));
         ++rc;
-        l = l * alpha + rs;
+        l = l * alpha + (rs + rcorr);
+        l32 = l32 * alpha + rs;
         m = m_use;
         first = false;
         if (flags & kLast) break;
@@ -983,7 +996,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (p.lse != nullptr)
           p.lse[(long long)bh * p.n + i] =
-              l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+              l32 > 0.f ? (m + __log2f(l32)) * 0.6931471805599453f : -INFINITY;
       }
       tc_fence_before();
       mbar_arrive(bar_o_free(X));

@@ -398,4 +398,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// 2^k for an integer-valued k <= 127, built from the exponent field (exact); 0 below
+// the normal range (k < -126, or k = -inf).
+__device__ __forceinline__ float exp2_int(float k) {
+  return k >= -126.0f ? __int_as_float(((int)k + 127) << 23) : 0.0f;
+}
+
 }  // namespace wise

@@ -21,3 +21,15 @@ def pytest_collection_modifyitems(config, items):
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
+
+
+def pytest_terminal_summary(terminalreporter):
+    # worst O error over every GPU-vs-oracle comparison of the session (flat bound 2e-2)
+    pu = sys.modules.get("parity_utils")
+    seen = getattr(pu, "O_OBSERVED", None) if pu else None
+    if seen:
+        mx = max(x[0] for x in seen)
+        mean = max(x[1] for x in seen)
+        terminalreporter.write_line(
+            f"O parity: {len(seen)} comparisons, worst max-abs {mx:.4e} (bound 2e-2), "
+            f"worst mean-abs {mean:.4e} (bound 2e-3)")

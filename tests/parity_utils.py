@@ -8,11 +8,11 @@ from oracle import wise_oracle as O
 from wise_inputs import bf16_bits_to_f64
 
 # Tolerances.
-#  * O: per element |err| <= 2e-2 + 2^-8 |O_ref|, and mean-abs 2e-3 per step (bf16
-#    inputs, fp32 accumulation).  The 2^-8 |O_ref| term is the rounding of the bf16
-#    output itself (unit roundoff of an 8-bit significand): rows that attend to a few
-#    keys have |O| near max |V|, where the absolute term alone would be tighter than
-#    the output's own rounding.
+#  * O: max-abs 2e-2 and mean-abs 2e-3 per compared output (bf16 inputs, fp32
+#    accumulation), flat, as the workload contract states them.  The output is bf16,
+#    so its own rounding already spends up to 2^-6 = 0.0156 where |O| is in [4, 8);
+#    the kernel keeps the rest small by normalising with the sum of the bf16 P it
+#    multiplies into V.
 #  * lse: 2e-3 absolute.  Scores are exact bf16 products summed in fp32 (relative
 #    error <= d * 2^-24 of sum |q_c k_c|, ~4e-4 in logit units at the largest logits
 #    of these workloads); the row sum of up to 16384 fp32 terms adds <= n * 2^-24
@@ -23,6 +23,8 @@ from wise_inputs import bf16_bits_to_f64
 #    1e-4 (cumulative mass at the cut or one block before it within 1e-4 of eta, or a
 #    differing block's mass within 1e-4 of the cut block's mass).
 O_MAX, O_MEAN = 2e-2, 2e-3
+# every compare_o of the session appends (max-abs, mean-abs); conftest prints the worst
+O_OBSERVED: list = []
 LSE_TOL = 2e-3
 MASS_TOL = 1e-4
 CUT_TOL = 1e-4
@@ -41,10 +43,9 @@ def compare_o(o_gpu: np.ndarray, o_ref: np.ndarray, what: str = "O"):
     err = np.abs(o_gpu.astype(np.float64) - o_ref)
     mx, mean = float(err.max()), float(err.mean())
     assert np.isfinite(o_gpu).all(), f"{what}: non-finite output"
-    excess = err - (O_MAX + 2.0 ** -8 * np.abs(o_ref))
-    assert excess.max() <= 0.0, (
-        f"{what}: max-abs {mx:.3e}, bound 2e-2 + 2^-8 |O| exceeded by {excess.max():.3e}")
+    assert mx <= O_MAX, f"{what}: max-abs {mx:.3e} > {O_MAX}"
     assert mean <= O_MEAN, f"{what}: mean-abs {mean:.3e} > {O_MEAN}"
+    O_OBSERVED.append((mx, mean))
     return mx, mean
 
 

@@ -11,8 +11,10 @@ Each role here is a generator that follows the kernel's sequence of arrivals and
 waits.  Waits use the hardware's parity semantics (try_wait.parity(i & 1) passes
 while the barrier's current phase has the other parity), so a wait that passes a
 phase early or late is an error.  TMA copies land after random delays; an MMA may
-read or write its operands at any moment between its issue and its completion,
-and a commit arrives when every earlier MMA has completed.  The model flags:
+read or write its operands at any moment between its issue and its completion, but
+not before an MMA issued earlier has touched its own (tcgen05 MMAs of one thread
+execute in issue order; ``mma_in_order=False`` drops that), and a commit arrives
+when every earlier MMA has completed.  The model flags:
 a buffer (Q, K stage, V stage, S/P, O) overwritten while a reader still needs it,
 an MMA or the softmax reading the wrong generation of a buffer, an early or late
 phase, a deadlock, and a tile whose output misses entries.
@@ -44,8 +46,10 @@ class Bar:
             self.pending = self.count
 
 class Sim:
-    def __init__(self, seed, tiles_per_cta_list, mode, NK, NV, R=4, drop=()):
+    def __init__(self, seed, tiles_per_cta_list, mode, NK, NV, R=4, drop=(), mma_in_order=True):
         self.drop = frozenset(drop)
+        self.mma_in_order = mma_in_order
+        self.last_effect = 0
         self.rng = random.Random(seed)
         self.mode = mode  # 'attn' or 'mass'
         self.attn = mode == 'attn'
@@ -101,8 +105,10 @@ class Sim:
         op['done'] = start + dur
         self.mma_busy_until = op['done']
         self.inflight.append(op)
-        # effects at a random time in [issue, done]
-        te = self.rng.randint(self.t, op['done'])
+        # effects at a random time in [issue, done], after the previous op's effects
+        lo = max(self.t, self.last_effect) if self.mma_in_order else self.t
+        te = self.rng.randint(lo, op['done'])
+        self.last_effect = te
         self.seq += 1
         self.events.append((te, self.seq, lambda op=op: self.mma_effect(op)))
         self.seq += 1
@@ -124,8 +130,8 @@ class Sim:
                 self.errors.append(f"QK g={g} reads Q[{x}]={self.Q[x]} want {op['tile']}")
             # S_X must not hold a P still needed
             cur = self.S[x]
-            if cur is not None and cur[0] == 'P' and cur[1] not in self.pv_done:
-                self.errors.append(f"QK g={g} overwrites P of g={cur[1]} before its PV completed")
+            if cur is not None and cur[0] == 'P' and cur[1] not in self.pv_read:
+                self.errors.append(f"QK g={g} overwrites P of g={cur[1]} before its PV read it")
             if cur is not None and cur[0] == 'S' and cur[1] not in self.s_read:
                 self.errors.append(f"QK g={g} overwrites S of g={cur[1]} before it was read")
             self.S[x] = ('S', g)
@@ -135,6 +141,7 @@ class Sim:
                 self.errors.append(f"PV g={g} reads V stage holding {self.Vst.get(g % self.NV)}")
             if self.S[x] != ('P', g):
                 self.errors.append(f"PV g={g} reads S[{x}]={self.S[x]}")
+            self.pv_read.add(g)
             if op['first']:
                 if self.O[x] is not None and self.O[x][0] != 'read':
                     self.errors.append(f"PV g={g} (first) overwrites unread O[{x}]={self.O[x]}")
@@ -278,11 +285,10 @@ class Sim:
                 yield from issue_pv(x)
             if e['kind'] == 'end':
                 st['ended'] = True; return
-            if st['qkc'] >= 1:
-                if self.attn:
-                    yield self.wait(('o_done', x), st['pvc'] - 1)
-                else:
-                    yield self.wait(('s_free', x), st['qkc'] - 1)
+            # attention: S_X holds the P that the PV just issued reads; in-order MMA
+            # execution lets this QK follow it without a wait
+            if st['qkc'] >= 1 and not self.attn:
+                yield self.wait(('s_free', x), st['qkc'] - 1)
             self.mma_issue(dict(kind='QK', x=x, g=g, tile=e['tile']))
             self.mma_commit(('s_full', x))
             self.mma_commit(('k_empty', ks))
@@ -357,7 +363,7 @@ class Sim:
 
     # ------------------------------------------------------------ driver
     def run(self):
-        self.pv_done, self.qk_done, self.s_read = set(), set(), set()
+        self.pv_done, self.qk_done, self.s_read, self.pv_read = set(), set(), set(), set()
         self.tile_gs = {}
         roles = {'prod': self.producer(), 'v': self.vproducer(), 'mma': self.issuer(),
                  'sm0': self.softmax(0), 'sm1': self.softmax(1)}
@@ -425,7 +431,7 @@ def make_tiles(rng, ntiles):
     return out
 
 
-def run_seeds(seeds, drop=()):
+def run_seeds(seeds, drop=(), mma_in_order=True):
     """Run the model over random tile mixes; returns {seed: errors} for failing runs."""
     bad = {}
     for seed in seeds:
@@ -435,7 +441,7 @@ def run_seeds(seeds, drop=()):
         NK = rng.choice([3, 4, 6]) if mode == 'mass' else rng.choice([2, 3, 4])
         NV = rng.choice([2, 4]) if mode == 'attn' else 1
         tiles = make_tiles(rng, ntiles)
-        sim = Sim(seed, tiles, mode, NK, NV, drop=drop)
+        sim = Sim(seed, tiles, mode, NK, NV, drop=drop, mma_in_order=mma_in_order)
         try:
             errs = sim.run()
         except (AssertionError, IndexError, KeyError, TypeError) as exc:

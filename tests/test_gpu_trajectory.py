@@ -17,8 +17,8 @@ import numpy as np
 import pytest
 
 from oracle import wise_oracle as O
-from parity_utils import (MASS_TOL, bits_to_bool, check_csr, coarse_of_fine, compare_o,
-                          compare_selection)
+from parity_utils import MASS_TOL, bits_to_bool, check_csr, compare_o, compare_selection
+from traj_oracle import check_heads
 from wise_inputs import CONFIGS, bf16_bits_to_f64, iter_steps
 from wise_inputs.generator import StepPool
 
@@ -30,12 +30,16 @@ def _dev(bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
 
 
-def run_config(cfg, sample, check_steps, etas=(None,), block=32):
-    """Run all heads of `cfg` on the GPU; return host copies for the sampled heads."""
+def run_config(cfg, sel_heads, o_heads, o_steps, etas=(None,), block=32):
+    """Run all heads of `cfg` on the GPU; return host copies for the checked heads:
+    window-step masses / selections, union and schedule for `sel_heads`, and O at
+    `o_steps` for `o_heads`."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from recurrent_depth_lm_b200 import WiseTrajectory, ops
-    idx = [b * cfg.heads + h for (b, h) in sample]
+    heads = sorted(set(sel_heads) | set(o_heads))
+    idx = [b * cfg.heads + h for (b, h) in heads]
+    oi = [heads.index(x) for x in o_heads]
     trajs = {eta: WiseTrajectory(cfg.batch, cfg.heads, cfg.seqlen, cfg.head_dim, t_d=cfg.t_d,
                                  window=cfg.window, eta=cfg.eta if eta is None else eta,
                                  block=block, keep_step_bits=True) for eta in etas}
@@ -47,83 +51,70 @@ def run_config(cfg, sample, check_steps, etas=(None,), block=32):
             for eta, tr in trajs.items():
                 o = tr.step(t, dq, dk, dv)
                 flat = lambda x: x.reshape(cfg.bh, *x.shape[2:])[idx]
-                if t in check_steps:
+                if t in o_steps:
                     res[eta]["o"][t] = flat(o).float().cpu().numpy()
                 if tr.in_window(t):
                     res[eta]["mass"][t] = flat(tr.mass).cpu().numpy()
                     res[eta]["bits"][t] = flat(tr.step_bits[t]).cpu().numpy()
     torch.cuda.synchronize()
     assert ops.device_status() == 0
+    jobs = {}
     for eta, tr in trajs.items():
         ro = tr.row_offsets.cpu().numpy()
         ci = tr.col_idx.cpu().numpy()
         nq = cfg.nq
-        res[eta]["union"] = tr.union.reshape(cfg.bh, nq, -1)[idx].cpu().numpy()
-        res[eta]["sched"] = [(ro[i * nq:(i + 1) * nq + 1] - ro[i * nq],
-                              ci[ro[i * nq]:ro[(i + 1) * nq]]) for i in idx]
-        res[eta]["density"] = tr.density()
-    return res
-
-
-def check_config(cfg, sample, check_steps, etas=(None,), block=32):
-    res = run_config(cfg, sample, check_steps, etas, block)
-    f = block // 32
-    nq = cfg.nq
-    host = {t: (q, k, v) for t, q, k, v in iter_steps(cfg, heads=sample)}
-    report = {}
-    for eta in etas:
+        union = tr.union.reshape(cfg.bh, nq, -1)[idx].cpu().numpy()
         r = res[eta]
-        e = cfg.eta if eta is None else eta
-        exempt = 0
-        for si in range(len(sample)):
-            # window steps: mass and selection
-            step_sel = []
-            for t in range(cfg.window[0], cfg.window[1] + 1):
-                q, k, _ = (bf16_bits_to_f64(x[si]) for x in host[t])
-                r_ref = O.block_mass(q, k, cfg.scale)
-                assert np.abs(np.tril(r["mass"][t][si]) - r_ref).max() <= MASS_TOL
-                sel_gpu = bits_to_bool(r["bits"][t][si], nq)
-                if f == 1:
-                    exempt += compare_selection(sel_gpu, r_ref, e)
-                else:   # block-size variant: coarse selection, run as 32 x 32 subtiles
-                    coarse = coarse_of_fine(sel_gpu, f)
-                    assert np.array_equal(sel_gpu, O.expand_support(coarse, f))
-                    exempt += compare_selection(coarse, O.block_mass(q, k, cfg.scale, block), e)
-                step_sel.append(sel_gpu)
-            union = bits_to_bool(r["union"][si], nq)
-            assert np.array_equal(union, O.temporal_union(step_sel))
-            ro, ci = r["sched"][si]
-            check_csr(ro, ci, union)
-            sup = O.support_from_csr(ro, ci, nq)
-            for t in check_steps:
-                q, k, v = (bf16_bits_to_f64(x[si]) for x in host[t])
-                if t <= cfg.t_d:
-                    ref, _ = O.causal_attention(q, k, v, cfg.scale)
-                else:
-                    ref, _ = O.masked_attention(q, k, v, sup, cfg.scale)
-                    if e >= 1.0:   # eta = 1 reproduces dense causal attention
-                        dense, _ = O.causal_attention(q, k, v, cfg.scale)
-                        compare_o(r["o"][t][si], dense, f"eta=1 step {t}")
-                compare_o(r["o"][t][si], ref, f"{cfg.name} head {sample[si]} step {t}")
-        report[eta] = {"exempt_rows": exempt, "density": r["density"]}
+        jobs[eta] = []
+        for j, (hd, i) in enumerate(zip(heads, idx)):
+            gpu = {"mass": {t: m[j] for t, m in r["mass"].items()},
+                   "bits": {t: bb[j] for t, bb in r["bits"].items()},
+                   "union": union[j],
+                   "sched": (ro[i * nq:(i + 1) * nq + 1] - ro[i * nq],
+                             ci[ro[i * nq]:ro[(i + 1) * nq]]),
+                   "o": {t: o[j] for t, o in r["o"].items()} if j in oi else {}}
+            jobs[eta].append((cfg, hd, cfg.eta if eta is None else eta, block, gpu))
+        jobs[eta] = (jobs[eta], tr.density())
+    return jobs
+
+
+def check_config(cfg, sel_heads, o_heads, o_steps, etas=(None,), block=32):
+    """Returns {eta: {"exempt_rows", "density", "o_max", "heads"}}; prints the counts."""
+    jobs = run_config(cfg, sel_heads, o_heads, o_steps, etas, block)
+    report = {}
+    for eta, (js, density) in jobs.items():
+        out = check_heads(js)
+        o_max = max((x[1] for r in out for x in r["o"]), default=0.0)
+        report[eta] = {"exempt_rows": sum(r["exempt"] for r in out), "density": density,
+                       "o_max": o_max, "heads": len(out)}
+        print(f"{cfg.name} eta={eta or cfg.eta} block={block}: {len(out)} heads checked, "
+              f"{report[eta]['exempt_rows']} near-cut rows exempt, worst O max-abs "
+              f"{o_max:.3e}, density {density:.4f}")
     return report
+
+
+def all_heads(cfg):
+    return [(b, h) for b in range(cfg.batch) for h in range(cfg.heads)]
 
 
 def test_trajectory_tiny_all_heads_all_steps():
     cfg = CONFIGS["tiny"]
-    rep = check_config(cfg, [(0, 0), (0, 1)], check_steps=range(1, cfg.steps + 1))
+    rep = check_config(cfg, all_heads(cfg), all_heads(cfg), range(1, cfg.steps + 1))
     assert rep[None]["exempt_rows"] <= 1
 
 
 def test_trajectory_1k():
     cfg = CONFIGS["1k"]
-    check_config(cfg, [(0, 0), (0, 13), (0, 31)], check_steps=range(1, cfg.steps + 1))
+    rep = check_config(cfg, all_heads(cfg), [(0, 0), (0, 13), (0, 22), (0, 31)],
+                       range(1, cfg.steps + 1))
+    # 32 heads x 32 query blocks x 4 window steps = 4096 selection rows
+    assert rep[None]["exempt_rows"] <= 8
 
 
 @pytest.mark.parametrize("block", [64, 128])
 def test_trajectory_1k_block_sizes(block):
     cfg = CONFIGS["1k"]
-    rep = check_config(cfg, [(0, 0), (0, 31)], check_steps=[12, 13, 32], block=block)
+    rep = check_config(cfg, [(0, 0), (0, 31)], [(0, 0), (0, 31)], [12, 13, 32], block=block)
     assert rep[None]["exempt_rows"] <= 2
 
 
@@ -140,23 +131,35 @@ VARIANTS = [
 def test_trajectory_1k_hyperparameter_variants(variant):
     cfg = CONFIGS["1k"].with_(**variant)
     late = [cfg.t_d + 1, cfg.steps]
-    rep = check_config(cfg, [(0, 3), (0, 30)], check_steps=late)
+    rep = check_config(cfg, [(0, 3), (0, 30)], [(0, 3), (0, 30)], late)
     assert rep[None]["exempt_rows"] <= 2
 
 
 def test_trajectory_4k():
     cfg = CONFIGS["4k"]
-    check_config(cfg, [(0, 0), (0, 21)], check_steps=[1, 9, 12, 13, 20, 32])
+    # every head's window-step masses and selections (32 x 128 x 4 = 16384 rows); O on 4
+    rep = check_config(cfg, all_heads(cfg), [(0, 0), (0, 11), (0, 21), (0, 31)],
+                       [1, 9, 12, 13, 20, 32])
+    assert rep[None]["exempt_rows"] <= 16
 
 
 def test_trajectory_2k_b4_h40_d96():
     cfg = CONFIGS["2k_b4_h40_d96"]
-    check_config(cfg, [(0, 0), (2, 17), (3, 39)], check_steps=[1, 12, 13, 25, 32])
+    # every head of every batch (160 x 64 x 4 = 40960 selection rows); O on 5 heads,
+    # including the last head of the last batch
+    rep = check_config(cfg, all_heads(cfg), [(0, 0), (1, 20), (2, 17), (3, 0), (3, 39)],
+                       [1, 12, 13, 25, 32])
+    assert rep[None]["exempt_rows"] <= 40
 
 
 def test_trajectory_16k_and_eta_one():
     cfg = CONFIGS["16k"]
-    check_config(cfg, [(0, 5)], check_steps=[12, 13, 32], etas=(None, 1.0))
+    # 8 heads' window-step masses and selections (8 x 512 x 4 = 16384 rows); O on 4
+    sel = [(0, h) for h in (0, 5, 9, 14, 18, 23, 27, 31)]
+    rep = check_config(cfg, sel, [(0, 5), (0, 14), (0, 23), (0, 31)], [12, 13, 32],
+                       etas=(None, 1.0))
+    assert rep[None]["exempt_rows"] <= 16
+    assert rep[1.0]["exempt_rows"] == 0 and rep[1.0]["density"] == 1.0
 
 
 # ------------------------------------------------------------- selection-only controls

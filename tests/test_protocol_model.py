@@ -21,3 +21,11 @@ def test_each_wait_is_needed(bar):
     """Skipping the waits on one barrier makes the model report a hazard, a wrong phase, a
     broken invariant or a deadlock for some tile mix (a planted protocol mistake)."""
     assert run_seeds(range(600), drop={bar}), f"dropping the {bar} waits went unnoticed"
+
+
+def test_issue_order_is_what_lets_qk_follow_pv():
+    """The issuer starts a slot's next QK right after the PV that reads the slot's P,
+    without waiting for that PV: if MMAs could touch their operands out of issue order,
+    the model would see the QK overwrite P before the PV read it."""
+    bad = run_seeds(range(600), mma_in_order=False)
+    assert any("before its PV read it" in e for errs in bad.values() for e in errs)
