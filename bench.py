@@ -117,6 +117,21 @@ def sparse_flops(cfg, row_offsets, col_idx) -> float:
     return 4.0 * cfg.head_dim * pairs
 
 
+def tile_waste(cfg, row_offsets, col_idx):
+    """(issued, selected) 32x32 block units of a schedule.  A 128-row tile runs every key
+    block that any of its 4 query blocks keeps, for all 4 of them, so it issues
+    4 * |union of the 4 rows| block units against the rows' own counts."""
+    import numpy as np
+    nq = cfg.nq
+    ro = np.asarray(row_offsets, np.int64)
+    ci = np.asarray(col_idx, np.int64)[: ro[-1]]
+    nrows = len(ro) - 1
+    rows = np.repeat(np.arange(nrows), np.diff(ro))
+    tiles = (rows // nq) * ((nq + 3) // 4) + (rows % nq) // 4
+    pairs = np.unique(tiles * nq + ci)          # distinct (tile, key block)
+    return 4 * len(pairs), len(ci)
+
+
 # ------------------------------------------------------------------ measurement helpers
 
 def load_peaks():
@@ -294,6 +309,102 @@ class TrajectoryRunner:
                 if events is not None:
                     events.setdefault("sparse", []).append((a, ev()))
         return self.o
+
+
+def all_blocks_schedule(cfg, device):
+    """The CSR schedule of every causal block (the matched comparison's support)."""
+    import torch
+    from recurrent_depth_lm_b200 import ops
+    full = torch.full((cfg.batch, cfg.heads, cfg.nq, ops.words_per_row(cfg.nq)), -1,
+                      dtype=torch.int32, device=device)
+    ro, ci, _ = ops.build_schedule(full, head_dim=cfg.head_dim, exact_nnz=False)
+    return ro, ci
+
+
+def late_step_us(cfg, q, k, v, ro, ci, o, reps: int = 1):
+    """Median CUDA-event time of the block-sparse kernel over the late steps' inputs."""
+    import torch
+    from recurrent_depth_lm_b200 import ops
+    xs = []
+    for _ in range(reps):
+        for t in range(cfg.t_d + 1, cfg.steps + 1):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            ops.sparse_attn(q[t - 1], k[t - 1], v[t - 1], ro, ci, ci.numel(), o=o)
+            b.record()
+            xs.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.median(x.elapsed_time(y) * 1000.0 for x, y in xs)
+
+
+def matched_record(cfg, q, k, v, runner, device, f_sparse):
+    """The late step on the WISE schedule against the same kernel on every causal block
+    (the pages' matched exact-B=32 comparison), with density and tile waste."""
+    import numpy as np
+    tr = runner.traj
+    ro_w, ci_w = tr.row_offsets, tr.col_idx
+    ro_a, ci_a = all_blocks_schedule(cfg, device)
+    late_us_w = late_step_us(cfg, q, k, v, ro_w, ci_w, runner.o, reps=2)
+    late_us_a = late_step_us(cfg, q, k, v, ro_a, ci_a, runner.o, reps=2)
+    issued, selected = tile_waste(cfg, ro_w.cpu().numpy(), ci_w.cpu().numpy())
+    density = tr.density()
+    return {"late_step_us": round(late_us_w, 2),
+            "all_blocks_late_step_us": round(late_us_a, 2),
+            "speedup": round(late_us_a / late_us_w, 3),
+            "inverse_density": round(1.0 / density, 3),
+            "density": round(density, 4),
+            "issued_over_selected_blocks": round(issued / selected, 4),
+            "late_step_tflops": round(f_sparse / (late_us_w * 1e-6) / 1e12, 2)}
+
+
+def config_record(cfg, q, k, v, device, reps: int, peak: float):
+    """One workload measured on its own: per-call medians over `reps` trajectories, the
+    matched all-blocks late step and the tile waste."""
+    import torch
+    runner = TrajectoryRunner(cfg, device)
+    for _ in range(2):
+        runner.run(q, k, v)
+    torch.cuda.synchronize()
+    events = {}
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(reps):
+        runner.run(q, k, v, events=events)
+    t1.record()
+    torch.cuda.synchronize()
+    traj_us = t0.elapsed_time(t1) * 1000.0 / reps
+    med = {kind: statistics.median(a.elapsed_time(b) * 1000.0 for a, b in xs)
+           for kind, xs in events.items()}
+    ro = runner.traj.row_offsets.cpu().numpy()
+    ci = runner.traj.col_idx.cpu().numpy()
+    f_dense, f_sparse = dense_flops(cfg), sparse_flops(cfg, ro, ci)
+    traj_flops = cfg.t_d * f_dense + (cfg.steps - cfg.t_d) * f_sparse
+    late, dense = med.get("sparse"), med.get("dense")
+    rec = {"workload": f"{cfg.name}: batch {cfg.batch}, {cfg.heads} heads, head_dim "
+                       f"{cfg.head_dim}, n={cfg.seqlen}, eta={cfg.eta}",
+           "trajectory_us": round(traj_us, 1),
+           "trajectory_tflops": round(traj_flops / (traj_us * 1e-6) / 1e12, 2),
+           "late_step_us": round(late, 2),
+           "late_step_tflops": round(f_sparse / (late * 1e-6) / 1e12, 2),
+           "late_step_frac": round(f_sparse / (late * 1e-6) / 1e12 / peak, 4),
+           "dense_step_us": round(dense, 2) if dense else None,
+           "dense_step_tflops": round(f_dense / (dense * 1e-6) / 1e12, 2) if dense else None,
+           "dense_step_frac": round(f_dense / (dense * 1e-6) / 1e12 / peak, 4) if dense else None,
+           "window_step_us": round(med["dense_mass"], 2),
+           "select_us": round(med["select"], 2),
+           "schedule_us": round(med["schedule"], 2),
+           "setup_inclusive_late_us": round(((cfg.steps - cfg.t_d) * late + med["schedule"])
+                                            / (cfg.steps - cfg.t_d), 2),
+           "trajectories_timed": reps,
+           "l2": ("inputs fit in L2 (one trajectory is "
+                  f"{3 * cfg.steps * cfg.bh * cfg.seqlen * cfg.head_dim * 2 / 1e6:.1f} MB)"
+                  if 3 * cfg.steps * cfg.bh * cfg.seqlen * cfg.head_dim * 2 < 126e6
+                  else "inputs larger than L2")}
+    rec["matched"] = matched_record(cfg, q, k, v, runner, device, f_sparse)
+    rec["density"] = rec["matched"]["density"]
+    return rec
 
 
 def run_e2e(cfg, runner, host_q, host_k, host_v, reps: int):
@@ -481,6 +592,7 @@ def bench_wise(args):
     ms_local = t_start.elapsed_time(t_end) / args.steps
     ms = reduce_max(ms_local, device)
     status = ops.device_status()
+    launches = runner.launches_per_trajectory() * args.steps
 
     def avg_us(kind):
         xs = [a.elapsed_time(b) * 1000.0 for a, b in events.get(kind, [])]
@@ -515,6 +627,8 @@ def bench_wise(args):
 
     routing = (routing_stats(cfg, q, k, v, device, args.block)
                if args.routing and args.block != 16 else None)
+    matched = (matched_record(cfg, q, k, v, runner, device, f_sparse)
+               if args.block != 16 else None)
 
     e2e = None
     if args.e2e:
@@ -526,6 +640,31 @@ def bench_wise(args):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(e2e_s * 1e3, 3)}
         del hq, hk, hv
+
+    workloads = None
+    if args.configs and (args.block == 16 or world > 1):
+        workloads = {"skipped": "per-workload records are taken at block size 32 on one GPU"}
+    elif args.configs:
+        # every other workload (16K also at eta = 1 on the same inputs), then the
+        # supplementary sparse-regime one; the headline's inputs are freed first
+        from wise_inputs import CONFIGS, SUPPLEMENTARY
+        del q, k, v
+        runner = None
+        torch.cuda.empty_cache()
+        todo = [c for n, c in CONFIGS.items() if n != cfg.name] + list(SUPPLEMENTARY.values())
+        workloads = {}
+        for c in todo:
+            xq, xk, xv, _ = make_inputs(c, 0, device, workers)
+            workloads[c.name] = config_record(c, xq, xk, xv, device, args.config_reps, peak)
+            if c.name == "16k":
+                workloads["16k_eta1"] = config_record(c.with_(eta=1.0), xq, xk, xv, device,
+                                                      args.config_reps, peak)
+            del xq, xk, xv
+            torch.cuda.empty_cache()
+        if "4k_sparse" in workloads:
+            workloads["4k_sparse"]["note"] = (
+                "supplementary: the 4K workload with the hot-block bias raised from 3 to 7.5 "
+                "(a working set of ~40% of causal blocks); not one of the five configs")
 
     cpu = None
     if rank == 0 and world == 1 and args.cpu_baseline:
@@ -564,8 +703,10 @@ def bench_wise(args):
         "schedule_us": round(sched_us, 2) if sched_us else None,
         "density": round(density, 4), "nnz_blocks": nnz,
         "routing": routing,
+        "matched": matched,
+        "workloads": workloads,
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
-        "gpu_launches": runner.launches_per_trajectory() * args.steps,
+        "gpu_launches": launches,
         "device_status": status,
     }
     if rank == 0:
@@ -626,12 +767,17 @@ def main(argv=None):
                     help="discovery window (default: the last four steps up to t_d)")
     ap.add_argument("--workers", type=int, default=0)
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
-    ap.add_argument("--e2e-reps", type=int, default=2)
+    ap.add_argument("--e2e-reps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-heads", type=int, default=16)
     ap.add_argument("--no-clocks", dest="clocks", action="store_false")
     ap.add_argument("--no-routing", dest="routing", action="store_false",
                     help="skip the untimed density / retained-future-mass pass")
+    ap.add_argument("--no-configs", dest="configs", action="store_false",
+                    help="skip the per-workload records of the other configs (measured "
+                         "after the headline's timed region)")
+    ap.add_argument("--config-reps", type=int, default=3,
+                    help="trajectories timed per extra workload record")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

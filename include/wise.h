@@ -283,8 +283,11 @@ int wise_build_schedule(const uint32_t* union_bits, int32_t* row_offsets, int32_
  * Limit      : batch * heads * seqlen / 32 <= 1,048,576 schedule rows; larger
  *              shapes return WISE_ERR_WORKSPACE (use wise_build_schedule).
  * Set-up     : the first call on each device looks up the array's device
- *              address (with that device current); make that first call before
- *              any stream capture.
+ *              address (with that device current) and keeps it with the id of
+ *              the current CUDA context; a call in another context (a second
+ *              context on the device, or the primary context after
+ *              cudaDeviceReset) looks it up again.  Make the first call in each
+ *              context before any stream capture.
  * Sharing    : all calls on a device use the same array and it keeps the last
  *              call's contents (nothing in it needs clearing: every entry read
  *              is written first by the same call).  Calls whose kernels overlap

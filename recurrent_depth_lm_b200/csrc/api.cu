@@ -49,8 +49,16 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Per-device state.  The device address of a __device__ variable belongs to the
+// context the module was loaded into, so it is cached together with that context's id
+// (unique for the life of the process, and new after a primary-context reset) and
+// looked up again when the current context differs.
 struct DeviceInfo {
   bool init = false;
+  unsigned long long ctx = 0;
   int sms = 0;
   unsigned int* status = nullptr;
 };
@@ -64,14 +72,16 @@ int device_info(DeviceInfo** out) {
   if (dev < 0 || dev >= kMaxDevices) return fail(WISE_ERR_CUDA, "device index %d unsupported", dev);
   std::lock_guard<std::mutex> lk(g_dev_mu);
   DeviceInfo& di = g_dev[dev];
-  if (!di.init) {
+  unsigned long long ctx = 0;
+  const bool have_ctx = wise::current_context_id(&ctx);
+  if (!di.init || !have_ctx || di.ctx != ctx) {
     e = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, wise::g_status_word);
+    e = cudaGetSymbolAddress(&p, wise::g_status_word);   // creates the context if needed
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
     di.status = static_cast<unsigned int*>(p);
-    di.init = true;
+    di.init = wise::current_context_id(&di.ctx);   // without an id: look up on every call
   }
   *out = &di;
   return WISE_OK;
@@ -173,6 +183,26 @@ int launch_attn(int mode, const void* q, const void* k, const void* v, void* o,
 }  // namespace
 
 namespace wise {
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 // For entry points defined in other translation units of the library.
 int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
 int record_ok() { return ok(); }

@@ -7,7 +7,10 @@
 // that loads the library holds it until the process exits.  Host code cannot
 // use the array's name as a device address, so the first call on each device
 // looks the address up with cudaGetSymbolAddress (with that device current)
-// and caches it; make that first call before any stream capture.  All calls on
+// and caches it with the id of the current CUDA context; a call made in another
+// context (a second context on the device, or the primary context after a reset)
+// looks it up again.  Make the first call in a context before any stream
+// capture.  All calls on
 // a device share the one array and it keeps the previous call's contents: the
 // scan writes every entry it later reads, so nothing has to be cleared, but two
 // calls whose kernels overlap on the GPU (different streams, no ordering) race
@@ -30,10 +33,15 @@ constexpr long long kStaticMaxRows = kStaticScratchInts * kRowsPerScratchInt;  /
 static __device__ __align__(256) int g_sched_scratch[kStaticScratchInts];
 
 constexpr int kMaxDevices = 64;
-int* g_scratch_ptr[kMaxDevices] = {};
+struct ScratchAddr {
+  int* ptr = nullptr;
+  unsigned long long ctx = 0;   // id of the context ptr belongs to
+};
+ScratchAddr g_scratch[kMaxDevices];
 std::mutex g_scratch_mu;
 
-// Device address of g_sched_scratch on the current device (set up once per device).
+// Device address of g_sched_scratch in the current context (set up once per device and
+// context; without a context id, e.g. on a driver that lacks cuCtxGetId, on every call).
 int scratch_on_current_device(int** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -41,18 +49,23 @@ int scratch_on_current_device(int** out) {
   if (dev < 0 || dev >= kMaxDevices)
     return wise::record_error(WISE_ERR_CUDA, "device index out of range");
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  ScratchAddr& sa = g_scratch[dev];
+  unsigned long long ctx = 0;
+  const bool have_ctx = wise::current_context_id(&ctx);
+  if (sa.ptr == nullptr || !have_ctx || sa.ctx != ctx) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_sched_scratch);
+    e = cudaGetSymbolAddress(&p, g_sched_scratch);   // creates the context if needed
     if (e != cudaSuccess) {
       char msg[256];
       snprintf(msg, sizeof(msg), "cudaGetSymbolAddress(schedule scratch): %s",
                cudaGetErrorString(e));
       return wise::record_error(WISE_ERR_CUDA, msg);
     }
-    g_scratch_ptr[dev] = static_cast<int*>(p);
+    *out = static_cast<int*>(p);
+    sa.ptr = wise::current_context_id(&sa.ctx) ? *out : nullptr;
+    return WISE_OK;
   }
-  *out = g_scratch_ptr[dev];
+  *out = sa.ptr;
   return WISE_OK;
 }
 

@@ -81,5 +81,9 @@ int record_ok();
 int validate_shape(const wise_shape_t& s);
 // Device address of the current device's status word.
 int status_word(unsigned int** out);
+// Id of the calling thread's current CUDA context (unique for the life of the process;
+// a reset primary context gets a new one); false if there is none or the driver lacks
+// cuCtxGetId.
+bool current_context_id(unsigned long long* id);
 
 }  // namespace wise

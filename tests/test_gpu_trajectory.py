@@ -17,9 +17,10 @@ import numpy as np
 import pytest
 
 from oracle import wise_oracle as O
-from parity_utils import MASS_TOL, bits_to_bool, check_csr, compare_o, compare_selection
+from parity_utils import (MASS_TOL, O_OBSERVED, bits_to_bool, check_csr, compare_o,
+                          compare_selection)
 from traj_oracle import check_heads
-from wise_inputs import CONFIGS, bf16_bits_to_f64, iter_steps
+from wise_inputs import CONFIGS, SUPPLEMENTARY, bf16_bits_to_f64, iter_steps
 from wise_inputs.generator import StepPool
 
 pytestmark = pytest.mark.gpu
@@ -84,6 +85,7 @@ def check_config(cfg, sel_heads, o_heads, o_steps, etas=(None,), block=32):
     report = {}
     for eta, (js, density) in jobs.items():
         out = check_heads(js)
+        O_OBSERVED.extend((x[1], x[2]) for r in out for x in r["o"])   # worker comparisons
         o_max = max((x[1] for r in out for x in r["o"]), default=0.0)
         report[eta] = {"exempt_rows": sum(r["exempt"] for r in out), "density": density,
                        "o_max": o_max, "heads": len(out)}
@@ -150,6 +152,15 @@ def test_trajectory_2k_b4_h40_d96():
     rep = check_config(cfg, all_heads(cfg), [(0, 0), (1, 20), (2, 17), (3, 0), (3, 39)],
                        [1, 12, 13, 25, 32])
     assert rep[None]["exempt_rows"] <= 40
+
+
+def test_trajectory_4k_sparse_regime():
+    """The supplementary 4K workload with a ~40% working set (hot-block bias 7.5)."""
+    cfg = SUPPLEMENTARY["4k_sparse"]
+    rep = check_config(cfg, all_heads(cfg), [(0, 0), (0, 7), (0, 21), (0, 31)],
+                       [12, 13, 20, 32])
+    assert rep[None]["exempt_rows"] <= 16
+    assert 0.25 < rep[None]["density"] < 0.65
 
 
 def test_trajectory_16k_and_eta_one():

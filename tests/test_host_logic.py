@@ -95,6 +95,27 @@ def test_bench_flops_b16_counts_pairs_inside_kept_blocks():
     assert flops == 4.0 * cfg.head_dim * (256 + 136)
 
 
+def test_bench_tile_waste_counts_the_union_of_four_query_blocks():
+    """A 128-row tile issues every key block any of its 4 query blocks keeps, for all 4."""
+    import bench
+    from oracle import wise_oracle as O
+    from wise_inputs import CONFIGS
+    cfg = CONFIGS["tiny"].with_(heads=1)                # nq = 8: two tiles per head
+    full = np.tril(np.ones((8, 8), bool))
+    ro, ci = O.csr_schedule(full)
+    issued, selected = bench.tile_waste(cfg, ro, ci)
+    assert (issued, selected) == (4 * 4 + 4 * 8, 36)    # tiles run blocks 0-3 and 0-7
+    own = np.zeros((8, 8), bool)
+    own[4:, 0] = own[4:, 2] = True                      # rows 4-7 share one list
+    own[:4, 0] = True
+    own[1, 1] = True                                    # row 1 alone keeps block 1
+    ro, ci = O.csr_schedule(own)
+    assert bench.tile_waste(cfg, ro, ci) == (4 * 2 + 4 * 2, 4 + 1 + 8)
+    two = cfg.with_(heads=2)                            # heads never share a tile
+    ro2 = np.concatenate([ro, ro[1:] + ro[-1]])
+    assert bench.tile_waste(two, ro2, np.concatenate([ci, ci])) == (32, 26)
+
+
 def _fake_schedule(tr, rng):
     """A random causal working set and its CSR written into a CPU trajectory's buffers."""
     from oracle import wise_oracle as O
