@@ -529,8 +529,11 @@ def blas_threads() -> int:
 
 def workload(args):
     """The named workload with the one-at-a-time overrides (eta, t_d, window) applied."""
-    from wise_inputs import CONFIGS
-    cfg = CONFIGS[args.config]
+    from wise_inputs import CONFIGS, SUPPLEMENTARY
+    if args.config not in CONFIGS and args.config not in SUPPLEMENTARY:
+        raise SystemExit(f"unknown workload {args.config!r}: one of "
+                         f"{sorted(CONFIGS) + sorted(SUPPLEMENTARY)}")
+    cfg = CONFIGS.get(args.config) or SUPPLEMENTARY[args.config]
     kw = {}
     if args.eta is not None:
         kw["eta"] = args.eta
