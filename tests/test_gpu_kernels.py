@@ -765,3 +765,36 @@ def test_sparse_attn_b16_maximum_length(ops):
     o_ref, lse_ref = O.masked_attention(qf, kf, vf, sel, block=16)
     compare_o(dev_f32(o)[0, 0], o_ref, "B16 n=16384")
     assert np.abs(lse.cpu().numpy()[0, 0] - lse_ref).max() <= LSE_TOL
+
+
+@pytest.mark.parametrize("d", [64, 96])
+def test_maximum_length_dense_and_sparse(ops, d):
+    """n = 16384 (512 query blocks, 16 schedule words per row) at the head dims other than
+    128, with two query heads on one K/V head: dense attention with lse and the one-pass
+    block mass, and block-sparse attention with lse, each head against the oracle."""
+    b, h, hkv, n = 1, 2, 1, 16384
+    nq = n // 32
+    qb, _, _ = rand_qkv_bits(b, h, n, d, seed=16384 + d)
+    _, kb, vb = rand_qkv_bits(b, hkv, n, d, seed=16385 + d)
+    q, k, v = to_dev(qb), to_dev(kb), to_dev(vb)
+    o, lse, mass = ops.full_attn_mass(q, k, v, with_mass=True)
+    rng = np.random.default_rng(d)
+    sups = [random_support(nq, rng, p=0.3) for _ in range(b * h)]
+    ro, ci, nnz = csr_device(sups)
+    lse_s = torch.empty(b, h, n, device="cuda")
+    o_s, _ = ops.sparse_attn(q, k, v, ro, ci, nnz, lse=lse_s)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    o, lse, mass = dev_f32(o), lse.cpu().numpy(), mass.cpu().numpy()
+    o_s, lse_s = dev_f32(o_s), lse_s.cpu().numpy()
+    kf, vf = (bf16_bits_to_f64(x[0, 0]) for x in (kb, vb))
+    for hi in range(h):
+        qf = bf16_bits_to_f64(qb[0, hi])
+        o_ref, lse_ref = O.causal_attention(qf, kf, vf)
+        compare_o(o[0, hi], o_ref, f"dense n=16384 d={d} head {hi}")
+        assert np.abs(lse[0, hi] - lse_ref).max() <= LSE_TOL
+        if hi == 0:
+            assert np.abs(np.tril(mass[0, hi]) - O.block_mass(qf, kf)).max() <= MASS_TOL
+        o_ref, lse_ref = O.masked_attention(qf, kf, vf, sups[hi])
+        compare_o(o_s[0, hi], o_ref, f"sparse n=16384 d={d} head {hi}")
+        assert np.abs(lse_s[0, hi] - lse_ref).max() <= LSE_TOL
