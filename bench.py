@@ -253,10 +253,12 @@ class TrajectoryRunner:
     def launches_per_trajectory(self) -> int:
         cfg = self.cfg
         nwin = cfg.window[1] - cfg.window[0] + 1
-        # dense steps: 1 kernel; window steps: attention + mass + select; schedule: 3
+        # dense steps: 1 kernel; window steps: attention + fused mass/select at B = 32,
+        # attention + mass + select otherwise; schedule: 3
         # (block 16: 16-token mass + select; schedule fold + 3 + sub-masks = 5)
         sched = 5 if self.block == 16 else 3
-        return (cfg.t_d - nwin) + 3 * nwin + sched + (cfg.steps - cfg.t_d)
+        win = 2 if self.block == 32 else 3
+        return (cfg.t_d - nwin) + win * nwin + sched + (cfg.steps - cfg.t_d)
 
     def run(self, q, k, v, events=None):
         """One trajectory.  If `events` is a dict, append (start, end) event pairs per call kind."""
@@ -275,23 +277,26 @@ class TrajectoryRunner:
                 tr.step(t, q[t - 1], k[t - 1], v[t - 1], o=self.o)
                 if events is not None:
                     kind = ("sparse" if t > cfg.t_d else
-                            "dense_mass" if tr.in_window(t) else "dense")
+                            "window" if tr.in_window(t) else "dense")
                     events.setdefault(kind, []).append((a, ev()))
             return self.o
         for t in range(1, cfg.steps + 1):
             qt, kt, vt = q[t - 1], k[t - 1], v[t - 1]
             if t <= cfg.t_d:
-                if tr.in_window(t):
+                if tr.in_window(t) and self.block == 32:
+                    a = ev() if events is not None else None
+                    ops.window_step(qt, kt, vt, tr.union, cfg.eta, o=self.o, lse=tr.lse,
+                                    mass=tr.mass, workspace=tr.mass_ws)
+                    if events is not None:
+                        events.setdefault("window", []).append((a, ev()))
+                elif tr.in_window(t):
                     a = ev() if events is not None else None
                     ops.full_attn_mass(qt, kt, vt, o=self.o, lse=tr.lse, mass=tr.mass,
                                        workspace=tr.mass_ws)
-                    b = ev() if events is not None else None
                     ops.select_union(tr.mass, tr.union, cfg.eta, head_dim=cfg.head_dim,
                                      block=self.block)
-                    c = ev() if events is not None else None
                     if events is not None:
-                        events.setdefault("dense_mass", []).append((a, b))
-                        events.setdefault("select", []).append((b, c))
+                        events.setdefault("window", []).append((a, ev()))
                 else:
                     a = ev() if events is not None else None
                     ops.full_attn_mass(qt, kt, vt, o=self.o)
@@ -392,8 +397,8 @@ def config_record(cfg, q, k, v, device, reps: int, peak: float):
            "dense_step_us": round(dense, 2) if dense else None,
            "dense_step_tflops": round(f_dense / (dense * 1e-6) / 1e12, 2) if dense else None,
            "dense_step_frac": round(f_dense / (dense * 1e-6) / 1e12 / peak, 4) if dense else None,
-           "window_step_us": round(med["dense_mass"], 2),
-           "select_us": round(med["select"], 2),
+           "window_step_us": round(med["window"], 2),
+           "window_over_dense_us": round(med["window"] - dense, 2) if dense else None,
            "schedule_us": round(med["schedule"], 2),
            "setup_inclusive_late_us": round(((cfg.steps - cfg.t_d) * late + med["schedule"])
                                             / (cfg.steps - cfg.t_d), 2),
@@ -602,8 +607,7 @@ def bench_wise(args):
         return (statistics.median(xs), xs) if xs else (None, [])
 
     dense_us, _ = avg_us("dense")
-    dmass_us, _ = avg_us("dense_mass")
-    sel_us, _ = avg_us("select")
+    win_us, _ = avg_us("window")
     sched_us, _ = avg_us("schedule")
     sparse_us, sparse_all = avg_us("sparse")
     q25, q75 = (np.percentile(sparse_all, [25, 75]).tolist() if sparse_all else (None, None))
@@ -701,8 +705,9 @@ def bench_wise(args):
                                    if sparse_us and sched_us else None,
         "dense_step_us": round(dense_us, 2) if dense_us else None,
         "dense_step_tflops": round(f_dense / (dense_us * 1e-6) / 1e12, 2) if dense_us else None,
-        "window_step_us": round(dmass_us, 2) if dmass_us else None,
-        "select_us": round(sel_us, 2) if sel_us else None,
+        # a window step: attention + block mass + selection (two launches at B = 32)
+        "window_step_us": round(win_us, 2) if win_us else None,
+        "window_over_dense_us": round(win_us - dense_us, 2) if win_us and dense_us else None,
         "schedule_us": round(sched_us, 2) if sched_us else None,
         "density": round(density, 4), "nnz_blocks": nnz,
         "routing": routing,

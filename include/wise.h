@@ -12,6 +12,8 @@
  *                                  OR-ed into the working set; or
  *                                  wise_select_union_blocks for B = 64 / 128;
  *                                  the *_b16 calls for B = 16)
+ *                                wise_window_step      (a window step's attention,
+ *                                  block mass and selection in one call, B = 32)
  *   once, after step t_d       : wise_build_schedule   (CSR key-block schedule)
  *   late steps t > t_d         : wise_sparse_attn      (block-sparse attention)
  *   analysis, off the hot path : wise_select_size_matched / _mass_matched
@@ -101,6 +103,31 @@ typedef struct wise_shape {
 int wise_full_attn_mass(const void* q, const void* k, const void* v, void* o, float* lse,
                         float* mass, void* workspace, size_t workspace_bytes, wise_shape_t shape,
                         void* stream);
+
+/*
+ * One step of the discovery window in one call: dense causal attention with lse, the
+ * block mass and the step's cumulative-eta support ORed into the working set.
+ *
+ * Defines (WISE paper appendix B "WISE configuration": the window steps
+ * t_d - 3 .. t_d; section 3 recurrent attention equation; section 5.1 block mass;
+ * section 3 "attention support" and section 6.1 selection): exactly
+ *   wise_full_attn_mass(q, k, v, o, lse, mass, workspace, ...) followed by
+ *   wise_select_union(mass, union_bits, step_bits, eta, ...),
+ * with the same outputs bit for bit, in two launches: the attention kernel, which
+ * records every row's per-key-block log-sum-exp in `workspace`, and one kernel that
+ * forms the block masses of eight query blocks at a time and cuts each of their rows
+ * at eta from the masses it holds.
+ *
+ * q, k, v, o, lse, mass : as for wise_full_attn_mass; lse and mass are required.
+ * union_bits, step_bits, eta : as for wise_select_union.
+ * workspace  : device scratch of at least wise_mass_workspace_bytes(shape) bytes,
+ *              16-byte aligned (required).
+ * Errors     : WISE_ERR_ARG (a required pointer NULL, eta <= 0 or NaN), WISE_ERR_SHAPE,
+ *              WISE_ERR_ALIGN, WISE_ERR_WORKSPACE (too small), WISE_ERR_CUDA.
+ */
+int wise_window_step(const void* q, const void* k, const void* v, void* o, float* lse,
+                     float* mass, uint32_t* union_bits, uint32_t* step_bits, float eta,
+                     void* workspace, size_t workspace_bytes, wise_shape_t shape, void* stream);
 
 /* Workspace bytes of the one-pass block mass: B * H * nq * n * 4. */
 size_t wise_mass_workspace_bytes(wise_shape_t shape);

@@ -48,6 +48,8 @@ _SIGNATURES = {
     "wise_full_attn_mass": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
                                            WiseShape, _vp]),
     "wise_mass_workspace_bytes": (ctypes.c_size_t, [WiseShape]),
+    "wise_window_step": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float,
+                                        _vp, ctypes.c_size_t, WiseShape, _vp]),
     "wise_select_union": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_float, WiseShape, _vp]),
     "wise_select_union_blocks": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_float, ctypes.c_int32,
                                                 WiseShape, _vp]),
@@ -81,7 +83,7 @@ _SIGNATURES = {
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is not built; run `python -m recurrent_depth_lm_b200.build` "
+            f"{LIB_PATH} is not built; run `python recurrent_depth_lm_b200/build.py` "
             "(or __graft_entry__.build()) first. There is no non-CUDA fallback.")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in _SIGNATURES.items():

@@ -242,8 +242,9 @@ int wise_full_attn_mass(const void* q, const void* k, const void* v, void* o, fl
   rc = launch_attn(wise::kModeDense, q, k, v, o, p, shape, stream);
   if (rc) return rc;
   if (one_pass) {
-    cudaError_t e = wise::launch_mass_from_blse(p.blse, lse, mass, shape.batch * shape.heads,
-                                                shape.seqlen, static_cast<cudaStream_t>(stream));
+    cudaError_t e = wise::launch_mass_select(p.blse, lse, mass, nullptr, nullptr, 0.f,
+                                             shape.batch * shape.heads, shape.seqlen,
+                                             static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "mass launch");
   } else if (mass) {
     wise::AttnParams pm{};
@@ -252,6 +253,33 @@ int wise_full_attn_mass(const void* q, const void* k, const void* v, void* o, fl
     rc = launch_attn(wise::kModeMass, q, k, v, o, pm, shape, stream);
     if (rc) return rc;
   }
+  return ok();
+}
+
+int wise_window_step(const void* q, const void* k, const void* v, void* o, float* lse,
+                     float* mass, uint32_t* union_bits, uint32_t* step_bits, float eta,
+                     void* workspace, size_t workspace_bytes, wise_shape_t shape, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !lse || !mass || !union_bits || !workspace)
+    return fail(WISE_ERR_ARG, "q, k, v, o, lse, mass, union_bits and workspace must be non-NULL");
+  if (!(eta > 0.f)) return fail(WISE_ERR_ARG, "eta must be > 0 (got %g)", (double)eta);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(WISE_ERR_ALIGN, "q, k, v, o must be 16-byte aligned");
+  if (!aligned16(lse) || !aligned16(mass) || !aligned16(workspace))
+    return fail(WISE_ERR_ALIGN, "lse, mass and workspace must be 16-byte aligned");
+  const size_t need = wise_mass_workspace_bytes(shape);
+  if (workspace_bytes < need)
+    return fail(WISE_ERR_WORKSPACE, "mass workspace of %zu bytes required", need);
+  wise::AttnParams p{};
+  p.lse = lse;
+  p.blse = static_cast<float*>(workspace);
+  rc = launch_attn(wise::kModeDense, q, k, v, o, p, shape, stream);
+  if (rc) return rc;
+  cudaError_t e = wise::launch_mass_select(p.blse, lse, mass, union_bits, step_bits, eta,
+                                           shape.batch * shape.heads, shape.seqlen,
+                                           static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "mass/select launch");
   return ok();
 }
 

@@ -79,6 +79,30 @@ def full_attn_mass(q, k, v, *, with_mass: bool = False, o=None, lse=None, mass=N
     return o, lse, mass
 
 
+def window_step(q, k, v, union_bits, eta: float, *, step_bits=None, o=None, lse=None,
+                mass=None, workspace=None, scale=None, stream=None):
+    """One discovery-window step: dense attention, block mass and the eta-support ORed
+    into `union_bits` (in place), in one library call.  Returns (o, lse, mass)."""
+    b, h, n, d = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    kv = _check_qkv(q, k, v, o)
+    if mass is None:
+        mass = torch.empty(b, h, n // BLOCK, n // BLOCK, dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty(b, h, n, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = mass_workspace(b, h, n, d, q.device)
+    if mass.dtype != torch.float32 or union_bits.dtype != torch.int32:
+        raise ValueError("mass must be float32 and union_bits int32 (uint32 bit patterns)")
+    rc = lib.wise_window_step(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(mass),
+                              _ptr(union_bits), _ptr(step_bits), float(eta), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(),
+                              shape_of(q, scale, kv), _stream(stream))
+    check(rc, "wise_window_step")
+    return o, lse, mass
+
+
 def mass_workspace(b: int, h: int, n: int, head_dim: int, device) -> torch.Tensor:
     nbytes = lib.wise_mass_workspace_bytes(WiseShape(b, h, n, head_dim, 0.0))
     return torch.empty(max(1, nbytes // 4), dtype=torch.float32, device=device)

@@ -120,16 +120,23 @@ class WiseTrajectory:
                                      head_dim=self.d, stream=stream)
             elif self.in_window(t) or first:
                 m = self.mass1 if first else self.mass
-                o, _, _ = ops.full_attn_mass(q, k, v, o=o, lse=self.lse, mass=m,
-                                             workspace=self.mass_ws, scale=self.scale,
-                                             stream=stream)
-                if self.in_window(t):
-                    sb = None
-                    if self.keep_step_bits:
-                        sb = torch.empty_like(self.union)
-                        self.step_bits[t] = sb
-                    ops.select_union(m, self.union, self.eta, step_bits=sb, head_dim=self.d,
-                                     scale=self.scale, block=self.block, stream=stream)
+                sb = None
+                if self.in_window(t) and self.keep_step_bits:
+                    sb = torch.empty_like(self.union)
+                    self.step_bits[t] = sb
+                if self.in_window(t) and self.block == ops.BLOCK:
+                    # attention, block mass and selection in one library call
+                    o, _, _ = ops.window_step(q, k, v, self.union, self.eta, step_bits=sb, o=o,
+                                              lse=self.lse, mass=m, workspace=self.mass_ws,
+                                              scale=self.scale, stream=stream)
+                else:
+                    o, _, _ = ops.full_attn_mass(q, k, v, o=o, lse=self.lse, mass=m,
+                                                 workspace=self.mass_ws, scale=self.scale,
+                                                 stream=stream)
+                    if self.in_window(t):
+                        ops.select_union(m, self.union, self.eta, step_bits=sb,
+                                         head_dim=self.d, scale=self.scale, block=self.block,
+                                         stream=stream)
                 if first and self.support == "static95":
                     ops.select_union(m, self.control, self.eta, head_dim=self.d,
                                      scale=self.scale, block=self.block, stream=stream)

@@ -798,3 +798,46 @@ def test_maximum_length_dense_and_sparse(ops, d):
         o_ref, lse_ref = O.masked_attention(qf, kf, vf, sups[hi])
         compare_o(o_s[0, hi], o_ref, f"sparse n=16384 d={d} head {hi}")
         assert np.abs(lse_s[0, hi] - lse_ref).max() <= LSE_TOL
+
+
+# nq = 17 (a ragged group of query blocks), GQA, d = 96, and n = 16384 (16 mask words per row)
+WINDOW_SHAPES = [(1, 3, 544, 64, 3), (2, 4, 1024, 128, 2), (1, 2, 4096, 96, 1),
+                 (1, 1, 16384, 128, 1)]
+
+
+@pytest.mark.parametrize("b,h,n,d,hkv", WINDOW_SHAPES)
+def test_window_step_is_attention_mass_and_selection(ops, b, h, n, d, hkv):
+    """wise_window_step = wise_full_attn_mass + wise_select_union, bit for bit, ORing into
+    a working set from earlier steps; its masses and step support against the oracle."""
+    g, nq = h // hkv, n // 32
+    w = (nq + 31) // 32
+    qb, _, _ = rand_qkv_bits(b, h, n, d, seed=5 * n + h)
+    _, kb, vb = rand_qkv_bits(b, hkv, n, d, seed=5 * n + hkv + 1)
+    q, k, v = to_dev(qb), to_dev(kb), to_dev(vb)
+    eta = 0.9
+    rng = np.random.default_rng(n + d)
+    prior_np = (rng.integers(0, 2**32, (b, h, nq, w), dtype=np.uint64) &
+                rng.integers(0, 2**32, (b, h, nq, w), dtype=np.uint64) &
+                rng.integers(0, 2**32, (b, h, nq, w), dtype=np.uint64))
+    prior = torch.from_numpy(prior_np.astype(np.uint32).view(np.int32)).cuda()
+    u1, u2 = prior.clone(), prior.clone()
+    st1, st2 = torch.empty_like(prior), torch.empty_like(prior)
+    o1, lse1, m1 = ops.window_step(q, k, v, u1, eta, step_bits=st1)
+    o2, lse2, m2 = ops.full_attn_mass(q, k, v, with_mass=True)
+    ops.select_union(m2, u2, eta, step_bits=st2, head_dim=d)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    assert torch.equal(o1, o2) and torch.equal(lse1, lse2)
+    tri = torch.ones(nq, nq, dtype=torch.bool, device="cuda").tril()
+    assert torch.equal(m1[..., tri], m2[..., tri])
+    assert torch.equal(st1, st2) and torch.equal(u1, u2)
+    assert torch.equal(u1, prior | st1)
+    m1, st1 = m1.cpu().numpy(), st1.cpu().numpy()
+    exempt = 0
+    for bi, hi in sorted({(0, 0), (b - 1, h - 1)}):
+        qf = bf16_bits_to_f64(qb[bi, hi])
+        kf = bf16_bits_to_f64(kb[bi, hi // g])
+        r_ref = O.block_mass(qf, kf)
+        assert np.abs(np.tril(m1[bi, hi]) - r_ref).max() <= MASS_TOL
+        exempt += compare_selection(bits_to_bool(st1[bi, hi], nq), r_ref, eta)
+    assert exempt <= max(2, nq // 16)
