@@ -253,12 +253,10 @@ class TrajectoryRunner:
     def launches_per_trajectory(self) -> int:
         cfg = self.cfg
         nwin = cfg.window[1] - cfg.window[0] + 1
-        # dense steps: 1 kernel; window steps: attention + fused mass/select at B = 32,
-        # attention + mass + select otherwise; schedule: 3
+        # dense steps: 1 kernel; window steps: attention + mass + select; schedule: 3
         # (block 16: 16-token mass + select; schedule fold + 3 + sub-masks = 5)
         sched = 5 if self.block == 16 else 3
-        win = 2 if self.block == 32 else 3
-        return (cfg.t_d - nwin) + win * nwin + sched + (cfg.steps - cfg.t_d)
+        return (cfg.t_d - nwin) + 3 * nwin + sched + (cfg.steps - cfg.t_d)
 
     def run(self, q, k, v, events=None):
         """One trajectory.  If `events` is a dict, append (start, end) event pairs per call kind."""
@@ -705,7 +703,7 @@ def bench_wise(args):
                                    if sparse_us and sched_us else None,
         "dense_step_us": round(dense_us, 2) if dense_us else None,
         "dense_step_tflops": round(f_dense / (dense_us * 1e-6) / 1e12, 2) if dense_us else None,
-        # a window step: attention + block mass + selection (two launches at B = 32)
+        # a window step: attention + block mass + selection (three launches)
         "window_step_us": round(win_us, 2) if win_us else None,
         "window_over_dense_us": round(win_us - dense_us, 2) if win_us and dense_us else None,
         "schedule_us": round(sched_us, 2) if sched_us else None,

@@ -113,10 +113,9 @@ int wise_full_attn_mass(const void* q, const void* k, const void* v, void* o, fl
  * section 3 "attention support" and section 6.1 selection): exactly
  *   wise_full_attn_mass(q, k, v, o, lse, mass, workspace, ...) followed by
  *   wise_select_union(mass, union_bits, step_bits, eta, ...),
- * with the same outputs bit for bit, in two launches: the attention kernel, which
- * records every row's per-key-block log-sum-exp in `workspace`, and one kernel that
- * forms the block masses of eight query blocks at a time and cuts each of their rows
- * at eta from the masses it holds.
+ * with the same outputs bit for bit: the attention kernel records every row's
+ * per-key-block log-sum-exp in `workspace`, a light kernel turns them into block
+ * masses and the selection kernel cuts each row at eta.
  *
  * q, k, v, o, lse, mass : as for wise_full_attn_mass; lse and mass are required.
  * union_bits, step_bits, eta : as for wise_select_union.
@@ -140,7 +139,9 @@ size_t wise_mass_workspace_bytes(wise_shape_t shape);
  * admissible blocks b <= q are ranked by mass[bh][q][b], descending, ties to
  * the lower block index; the support is the shortest prefix whose cumulative
  * mass is >= eta.  If eta >= 1, or no prefix reaches eta, every admissible
- * block is kept.  Cumulative sums are taken in fp32.
+ * block is kept.  Masses are clamped to [0, 1]; cumulative sums are exact sums of
+ * the masses rounded to multiples of 2^-21, and a prefix reaches eta when that sum is
+ * at least ceil(eta * 2^21) * 2^-21 (so the result does not depend on summation order).
  *
  * mass       : fp32 [B, H, nq, nq] (entries b > q are not read).
  * union_bits : uint32 [B, H, nq, W], W = ceil(nq / 32), in/out.  Bit (b % 32)
@@ -165,7 +166,7 @@ int wise_select_union(const float* mass, uint32_t* union_bits, uint32_t* step_bi
  * query blocks q of Q and the fine key blocks b <= q of B of mass[bh][q][b]
  * (the block-mass equation of section 5.1 pooled exactly).  The coarse support
  * is chosen as in wise_select_union (rank descending, ties to the lower coarse
- * index, shortest prefix with cumulative mass >= eta, fp32 sums).  Fine row
+ * index, shortest prefix with cumulative mass >= eta, sums as there).  Fine row
  * q = Q F + a then keeps fine block b iff coarse block b / F is kept and b <= q.
  *
  * mass, union_bits, step_bits, eta : as for wise_select_union; the bit masks
@@ -232,12 +233,12 @@ int wise_sparse_attn_b16(const void* q, const void* k, const void* v, void* o,
  * wise_select_size_matched (SizeMatched): row (bh, q) keeps the K admissible blocks
  *   of largest mass, K = the number of set admissible bits of the reference row;
  *   ties go to the lower block index.  K = 0 gives an empty row.
- * wise_select_mass_matched (MassMatched): m = the fp32 sum of the masses of the
+ * wise_select_mass_matched (MassMatched): m = the sum of the masses of the
  *   reference row's set admissible blocks; the row keeps the cumulative-eta support
  *   at eta = m (rank descending, ties to the lower index, shortest prefix with
- *   cumulative fp32 mass >= m; m >= 1 keeps every admissible block).  The prefix
- *   sums use the same summation order as m, so a reference row that is itself a
- *   ranking prefix is reproduced exactly.  m = 0 gives an empty row.
+ *   cumulative mass >= m; m >= 1 keeps every admissible block).  m and the prefix
+ *   sums are the exact fixed-point sums of wise_select_union, so a reference row that
+ *   is itself a ranking prefix is reproduced exactly.  m = 0 gives an empty row.
  *
  * mass     : fp32 [B, H, nq, nq] (entries b > q are not read).
  * ref_bits : uint32 [B, H, nq, W] (bits b > q are ignored).

@@ -242,9 +242,8 @@ int wise_full_attn_mass(const void* q, const void* k, const void* v, void* o, fl
   rc = launch_attn(wise::kModeDense, q, k, v, o, p, shape, stream);
   if (rc) return rc;
   if (one_pass) {
-    cudaError_t e = wise::launch_mass_select(p.blse, lse, mass, nullptr, nullptr, 0.f,
-                                             shape.batch * shape.heads, shape.seqlen,
-                                             static_cast<cudaStream_t>(stream));
+    cudaError_t e = wise::launch_block_mass(p.blse, lse, mass, shape.batch * shape.heads,
+                                            shape.seqlen, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "mass launch");
   } else if (mass) {
     wise::AttnParams pm{};
@@ -276,10 +275,13 @@ int wise_window_step(const void* q, const void* k, const void* v, void* o, float
   p.blse = static_cast<float*>(workspace);
   rc = launch_attn(wise::kModeDense, q, k, v, o, p, shape, stream);
   if (rc) return rc;
-  cudaError_t e = wise::launch_mass_select(p.blse, lse, mass, union_bits, step_bits, eta,
-                                           shape.batch * shape.heads, shape.seqlen,
-                                           static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "mass/select launch");
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = wise::launch_block_mass(p.blse, lse, mass, shape.batch * shape.heads,
+                                          shape.seqlen, st);
+  if (e != cudaSuccess) return cuda_fail(e, "mass launch");
+  e = wise::launch_select_union(mass, union_bits, step_bits, eta, shape.batch * shape.heads,
+                                shape.seqlen / 32, st);
+  if (e != cudaSuccess) return cuda_fail(e, "select_union launch");
   return ok();
 }
 

@@ -1,5 +1,4 @@
-// mass.cu -- block mass from per-(row, key block) log-sum-exps, and the window step's
-// selection on the same rows (one-pass window steps).
+// mass.cu -- block mass from per-(row, key block) log-sum-exps (one-pass window steps).
 //
 // Wan & Chen, "Attention Routing Stabilizes Early: Working-Set Inference for
 // Recurrent-Depth Language Models", section 5.1: r_qb = (1/|I_q|) sum_{i in I_q}
@@ -9,40 +8,50 @@
 // final normaliser lse_i the inner sum is 2^(blse_ib - lse_i * log2 e).  This
 // kernel does the outer mean.
 //
-// One CTA per (bh, group of eight query blocks).  blse is [bh][key block][row], so
-// for one key block the group's 256 rows are 1 KB of contiguous memory: warp w takes
-// key blocks w, w + 8, ..., and each lane makes two 16-byte loads per key block
-// (rows 4 l .. 4 l + 3 of the group's first and second 128 rows); the eight lanes
-// that hold one query block's 32 rows sum them with three shuffles.  Only admissible
-// (row block, key block) pairs are read.  The group's mass rows collect in shared
-// memory; then warp j owns query block q0 + j: it writes that row of masses
-// (coalesced) and, in a window step, cuts the row at eta (section 3 "attention
-// support", section 6.1; eta_cut, as in select.cu) and ORs the support into the
-// working set (appendix B, "WISE configuration").
+// blse is [bh][key block][row], so for one key block the 256 rows of eight
+// consecutive query blocks are 1 KB of contiguous memory.  One warp takes one work
+// item: a (bh, group of eight query blocks, chunk of kChunk key blocks) tile of the
+// causal triangle.  Each lane issues all of the item's loads first (two 16-byte loads
+// per key block: rows 4 l .. 4 l + 3 of the group's first and second 128 rows), then
+// the eight lanes holding one query block's 32 rows sum them with three shuffles.
+// Items are numbered group by group, so every warp of the grid has the same short
+// chain of work and the whole causal triangle's loads are in flight at once.  Only
+// admissible (row block, key block) pairs are read or written.
 
 #include <cstdint>
 
-#include "select_cut.cuh"
 #include "sm100.cuh"
 #include "wise_internal.h"
 
 namespace wise {
 
 namespace {
-constexpr int kGroup = 8;   // query blocks per CTA, one warp each
+constexpr int kGroup = 8;                  // query blocks per item
+constexpr int kChunk = 4;                  // key blocks per item
+constexpr int kPerGroupRow = kGroup / kChunk;
+constexpr int kWarps = 8;                  // warps (items) per CTA
 constexpr float kLog2e = 1.4426950408889634f;
 }  // namespace
 
-template <int MAXW>
-__global__ void __launch_bounds__(kGroup * 32)
-    mass_select_kernel(const float* __restrict__ blse, const float* __restrict__ lse,
-                       float* __restrict__ mass, uint32_t* __restrict__ ubits,
-                       uint32_t* __restrict__ sbits, float eta, int n, int nq, int groups) {
-  extern __shared__ float rows_s[];   // [kGroup][nq] masses of the group's rows
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long bh = blockIdx.x / groups;
-  const int q0 = (int)(blockIdx.x % groups) * kGroup;
+// Items of one bh: group g (query blocks 8 g .. 8 g + 7) has kPerGroupRow * (g + 1) chunks,
+// covering key blocks 0 .. 8 g + 7; groups 0 .. g - 1 hold kPerGroupRow * g (g + 1) / 2.
+__global__ void __launch_bounds__(kWarps * 32)
+    block_mass_kernel(const float* __restrict__ blse, const float* __restrict__ lse,
+                      float* __restrict__ mass, int n, int nq, long long items_per_bh,
+                      long long items) {
+  const int lane = threadIdx.x & 31;
+  const long long item = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (item >= items) return;   // warp-uniform
+  const long long bh = item / items_per_bh;
+  const int it = (int)(item % items_per_bh);
+  int g = (int)((sqrtf(8.0f * (float)it / kPerGroupRow + 1.0f) - 1.0f) * 0.5f);
+  while (g > 0 && kPerGroupRow * g * (g + 1) / 2 > it) --g;
+  while (kPerGroupRow * (g + 1) * (g + 2) / 2 <= it) ++g;
+  const int c = it - kPerGroupRow * g * (g + 1) / 2;
+  const int q0 = g * kGroup;
   const int nrow = min(kGroup, nq - q0);
+  const int kb0 = c * kChunk;
+  const int kb_end = min(kb0 + kChunk, q0 + nrow);   // key blocks kb0 .. kb_end - 1
 
   // This lane's rows: 4 (lane % 8) .. + 3 of query block qa[h] = q0 + 4 h + lane / 8.
   int qa[2];
@@ -58,18 +67,29 @@ __global__ void __launch_bounds__(kGroup * 32)
       qa[h] = -1;   // past the last query block: never admissible
   }
   const float* base = blse + bh * nq * (long long)n + (long long)q0 * 32 + 4 * lane;
-  const int kb_end = q0 + nrow;
-#pragma unroll 2
-  for (int kb = warp; kb < kb_end; kb += kGroup) {   // warp-uniform trip count
-    const float* src = base + (long long)kb * n;
+  float4 x[kChunk][2];
+#pragma unroll
+  for (int u = 0; u < kChunk; ++u) {
+    const int kb = kb0 + u;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      x[u][h] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (kb < kb_end && qa[h] >= kb)
+        x[u][h] = __ldg(reinterpret_cast<const float4*>(base + (long long)kb * n + 128 * h));
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kChunk; ++u) {
+    const int kb = kb0 + u;
+    if (kb >= kb_end) break;   // warp-uniform
     float part[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       float a = 0.f;
       if (qa[h] >= kb) {
-        const float4 x = __ldg(reinterpret_cast<const float4*>(src + 128 * h));
-        a = (fast_exp2(fmaf(-l4[h].x, kLog2e, x.x)) + fast_exp2(fmaf(-l4[h].y, kLog2e, x.y))) +
-            (fast_exp2(fmaf(-l4[h].z, kLog2e, x.z)) + fast_exp2(fmaf(-l4[h].w, kLog2e, x.w)));
+        const float4 y = x[u][h];
+        a = (fast_exp2(fmaf(-l4[h].x, kLog2e, y.x)) + fast_exp2(fmaf(-l4[h].y, kLog2e, y.y))) +
+            (fast_exp2(fmaf(-l4[h].z, kLog2e, y.z)) + fast_exp2(fmaf(-l4[h].w, kLog2e, y.w)));
       }
       a += __shfl_xor_sync(0xffffffffu, a, 1);
       a += __shfl_xor_sync(0xffffffffu, a, 2);
@@ -79,69 +99,21 @@ __global__ void __launch_bounds__(kGroup * 32)
     if ((lane & 7) == 0) {
 #pragma unroll
       for (int h = 0; h < 2; ++h)
-        if (qa[h] >= kb) rows_s[(qa[h] - q0) * nq + kb] = part[h] * (1.0f / 32.0f);
+        if (qa[h] >= kb) mass[(bh * nq + qa[h]) * (long long)nq + kb] = part[h] * (1.0f / 32.0f);
     }
-  }
-  __syncthreads();
-  if (warp >= nrow) return;   // warp-uniform
-
-  const int q = q0 + warp;
-  const long long row = bh * nq + q;
-  const float* srow = rows_s + warp * nq;
-  float* mrow = mass + row * nq;
-  for (int kb = lane; kb <= q; kb += 32) mrow[kb] = srow[kb];
-  if (ubits == nullptr) return;
-
-  const int W = (nq + 31) >> 5;
-  float v[MAXW];
-  bool ok[MAXW];
-#pragma unroll
-  for (int s = 0; s < MAXW; ++s) {
-    const int kb = s * 32 + lane;
-    ok[s] = (s < W) && (kb <= q);
-    v[s] = ok[s] ? srow[kb] : 0.f;
-  }
-  bool sel[MAXW];
-  eta_cut<MAXW>(v, ok, eta, lane, sel);
-  uint32_t word = 0u;
-#pragma unroll
-  for (int s = 0; s < MAXW; ++s) {
-    const uint32_t w = __ballot_sync(0xffffffffu, sel[s]);
-    if (lane == s) word = w;
-  }
-  if (lane < W) {
-    const long long at = row * W + lane;
-    if (sbits != nullptr) sbits[at] = word;
-    ubits[at] |= word;
   }
 }
 
-cudaError_t launch_mass_select(const float* blse, const float* lse, float* mass,
-                               uint32_t* union_bits, uint32_t* step_bits, float eta, int BH,
-                               int n, cudaStream_t stream) {
+cudaError_t launch_block_mass(const float* blse, const float* lse, float* mass, int BH, int n,
+                              cudaStream_t stream) {
   const int nq = n / 32;
-  const int W = (nq + 31) / 32;
-  const int groups = (nq + kGroup - 1) / kGroup;
-  const long long ctas = (long long)BH * groups;
+  const long long groups = (nq + kGroup - 1) / kGroup;
+  const long long items_per_bh = kPerGroupRow * groups * (groups + 1) / 2;
+  const long long items = items_per_bh * BH;
+  const long long ctas = (items + kWarps - 1) / kWarps;
   if (ctas > 0x7fffffffLL) return cudaErrorInvalidValue;
-  const size_t smem = (size_t)kGroup * nq * sizeof(float);
-  const dim3 grid((unsigned)ctas), block(kGroup * 32);
-#define WISE_MASS_SELECT(MW)                                                                 \
-  mass_select_kernel<MW><<<grid, block, smem, stream>>>(blse, lse, mass, union_bits, step_bits, \
-                                                       eta, n, nq, groups)
-  if (W <= 1)
-    WISE_MASS_SELECT(1);
-  else if (W <= 2)
-    WISE_MASS_SELECT(2);
-  else if (W <= 4)
-    WISE_MASS_SELECT(4);
-  else if (W <= 8)
-    WISE_MASS_SELECT(8);
-  else if (W <= 16)
-    WISE_MASS_SELECT(16);
-  else
-    return cudaErrorInvalidValue;
-#undef WISE_MASS_SELECT
+  block_mass_kernel<<<(unsigned)ctas, kWarps * 32, 0, stream>>>(blse, lse, mass, n, nq,
+                                                               items_per_bh, items);
   return cudaGetLastError();
 }
 

@@ -9,7 +9,7 @@
 //
 // One warp per (bh, q) row.  Lane l holds the masses of blocks l, l+32, ...
 // so the selected set of word s is one __ballot_sync; the cut itself
-// (bisection over the float bit patterns, then ties in index order) is
+// (a radix select with exact fixed-point sums, then ties in index order) is
 // eta_cut in select_cut.cuh.
 
 #include <cstdint>
@@ -24,6 +24,7 @@ template <int MAXW>
 __global__ void __launch_bounds__(256)
     select_union_kernel(const float* __restrict__ mass, uint32_t* __restrict__ ubits,
                         uint32_t* __restrict__ sbits, float eta, long long rows, int nq) {
+  __shared__ __align__(16) uint32_t hist_s[8][256];   // eta_cut's digit histogram, per warp
   const int lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= rows) return;  // warp-uniform
@@ -41,7 +42,7 @@ __global__ void __launch_bounds__(256)
   }
 
   bool sel[MAXW];
-  eta_cut<MAXW>(v, ok, eta, lane, sel);
+  eta_cut<MAXW>(v, ok, eta, lane, sel, hist_s[threadIdx.x >> 5]);
 
   uint32_t word = 0u;
 #pragma unroll
@@ -67,6 +68,7 @@ template <int MAXWC, int F>
 __global__ void __launch_bounds__(256)
     select_union_pooled_kernel(const float* __restrict__ mass, uint32_t* __restrict__ ubits,
                                uint32_t* __restrict__ sbits, float eta, long long crows, int nq) {
+  __shared__ __align__(16) uint32_t hist_s[8][256];   // eta_cut's digit histogram, per warp
   const int lane = threadIdx.x & 31;
   const long long crow = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (crow >= crows) return;  // warp-uniform
@@ -95,7 +97,7 @@ __global__ void __launch_bounds__(256)
   }
 
   bool sel[MAXWC];
-  eta_cut<MAXWC>(v, ok, eta, lane, sel);
+  eta_cut<MAXWC>(v, ok, eta, lane, sel, hist_s[threadIdx.x >> 5]);
 
   // Fine word w covers fine blocks 32w .. 32w+31 = coarse blocks 32w/F .. (32w+31)/F,
   // all in coarse slot w / F; lane i's bit is the kept flag of coarse block (32w+i)/F.
@@ -265,14 +267,15 @@ __device__ __forceinline__ void store_bits_row(uint32_t* __restrict__ dst, int W
 }
 
 // kSize: SizeMatched, K_q = |W_q| blocks of largest mass.  kMass: MassMatched, the
-// cumulative-eta cut at eta = m_q, the mass of W_q, summed in the same order as the cut's
-// own sums (so a ranking prefix holding W_q's blocks reaches m_q exactly).
+// cumulative-eta cut at eta = m_q, the mass of W_q, in the cut's own fixed-point units
+// (so a ranking prefix holding W_q's blocks reaches m_q exactly).
 enum ControlKind { kSizeMatched = 0, kMassMatched = 1 };
 
 template <int MAXW, int KIND>
 __global__ void __launch_bounds__(256)
     select_control_kernel(const float* __restrict__ mass, const uint32_t* __restrict__ ref,
                           uint32_t* __restrict__ out, long long rows, int nq) {
+  __shared__ __align__(16) uint32_t hist_s[8][256];   // cut_at's digit histogram, per warp
   const int lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= rows) return;  // warp-uniform
@@ -293,18 +296,27 @@ __global__ void __launch_bounds__(256)
       topk_cut<MAXW>(v, ok, K, lane, sel);
     }
   } else {
-    const float m = warp_sum_ge<MAXW>(v, in, 0.f);
-    if (!(m > 0.f)) {
+    // m_q in the cut's units: the sum of the reference blocks' units, so a ranking
+    // prefix holding exactly W_q's blocks reaches it exactly
+    uint32_t part = 0u;
+#pragma unroll
+    for (int s = 0; s < MAXW; ++s) part += in[s] ? cut_units(v[s]) : 0u;
+    const uint32_t m = __reduce_add_sync(0xffffffffu, part);
+    if (m == 0u) {
 #pragma unroll
       for (int s = 0; s < MAXW; ++s) sel[s] = false;
+    } else if (m >= (uint32_t)kCutScale) {   // m_q >= 1 keeps every admissible block
+#pragma unroll
+      for (int s = 0; s < MAXW; ++s) sel[s] = ok[s];
     } else {
-      eta_cut<MAXW>(v, ok, m, lane, sel);
+      cut_at<MAXW>(v, ok, m, lane, sel, hist_s[threadIdx.x >> 5]);
     }
   }
   store_bits_row<MAXW>(out + row * W, W, lane, sel);
 }
 
-// retained[row] = sum of mass[row][b] over set bits b <= q (fp32, same order as above).
+// retained[row] = sum of mass[row][b] over set bits b <= q (fp32: per lane, then a
+// butterfly over the lanes).
 template <int MAXW>
 __global__ void __launch_bounds__(256)
     support_mass_kernel(const float* __restrict__ mass, const uint32_t* __restrict__ bits,
@@ -318,8 +330,12 @@ __global__ void __launch_bounds__(256)
   bool ok[MAXW], in[MAXW];
   load_mass_row<MAXW>(mass + row * (long long)nq, q, W, lane, v, ok);
   load_bits_row<MAXW>(bits + row * W, ok, lane, in);
-  const float m = warp_sum_ge<MAXW>(v, in, 0.f);
-  if (lane == 0) retained[row] = m;
+  float a = 0.f;
+#pragma unroll
+  for (int s = 0; s < MAXW; ++s) a += in[s] ? v[s] : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+  if (lane == 0) retained[row] = a;
 }
 
 // Calls f(std::integral_constant<int, MAXW>) for the smallest MAXW in {1, 2, 4, 8, 16} >= W.

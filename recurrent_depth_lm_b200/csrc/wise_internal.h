@@ -40,12 +40,9 @@ cudaError_t launch_attention(int mode, int d, const CUtensorMap& tq, const CUten
 int attention_smem_bytes(int mode, int d);
 
 // mass[bh][q][b] = (1/32) sum_{i in q} 2^(blse[bh][b][i] - lse[bh][i] * log2 e), b <= q
-// Block mass from the recorded per-(row, key block) log-sum-exps; with union_bits
-// non-NULL also the cumulative-eta support of every mass row, ORed into union_bits
-// (and written to step_bits if non-NULL).
-cudaError_t launch_mass_select(const float* blse, const float* lse, float* mass,
-                               uint32_t* union_bits, uint32_t* step_bits, float eta, int BH,
-                               int n, cudaStream_t stream);
+// Block mass from the recorded per-(row, key block) log-sum-exps.
+cudaError_t launch_block_mass(const float* blse, const float* lse, float* mass, int BH, int n,
+                              cudaStream_t stream);
 
 cudaError_t launch_select_union(const float* mass, uint32_t* union_bits, uint32_t* step_bits,
                                 float eta, int BH, int nq, cudaStream_t stream);
