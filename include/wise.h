@@ -139,9 +139,10 @@ size_t wise_mass_workspace_bytes(wise_shape_t shape);
  * admissible blocks b <= q are ranked by mass[bh][q][b], descending, ties to
  * the lower block index; the support is the shortest prefix whose cumulative
  * mass is >= eta.  If eta >= 1, or no prefix reaches eta, every admissible
- * block is kept.  Masses are clamped to [0, 1]; cumulative sums are exact sums of
- * the masses rounded to multiples of 2^-21, and a prefix reaches eta when that sum is
- * at least ceil(eta * 2^21) * 2^-21 (so the result does not depend on summation order).
+ * block is kept.  Masses are clamped to [0, 1] (NaN counts as 0); cumulative sums
+ * are exact sums of the masses rounded to multiples of 2^-21, and a prefix reaches
+ * eta when that sum is at least ceil(eta * 2^21) * 2^-21 (so the result does not
+ * depend on summation order).
  *
  * mass       : fp32 [B, H, nq, nq] (entries b > q are not read).
  * union_bits : uint32 [B, H, nq, W], W = ceil(nq / 32), in/out.  Bit (b % 32)

@@ -6,11 +6,11 @@
 // (descending, ties to the lower block index) whose cumulative mass reaches eta.
 // Used by every selection kernel of select.cu.
 //
-// Arithmetic.  Each mass is clamped to [0, 1] and rounded to the nearest multiple of
-// 2^-21; cumulative sums are then exact integer sums (a row holds at most 1024 masses,
-// so no sum exceeds 2^31), the same in any order, and a prefix reaches eta when its
-// sum is at least ceil(eta * 2^21).  The ranking uses the clamped fp32 masses
-// themselves.
+// Arithmetic.  Each mass is clamped to [0, 1] (NaN counts as 0) and rounded to the
+// nearest multiple of 2^-21; cumulative sums are then exact integer sums (a row holds
+// at most 1024 masses, so no sum exceeds 2^31), the same in any order, and a prefix
+// reaches eta when its sum is at least ceil(eta * 2^21).  The ranking uses the clamped
+// fp32 masses themselves.
 //
 // Method.  Lane l holds the masses of blocks s * 32 + l.  The cut value tau (the
 // smallest mass of the shortest prefix) is found by a most-significant-digit radix
@@ -48,7 +48,7 @@ __device__ __forceinline__ void cut_at(const float (&v)[MAXW], const bool (&ok)[
   uint32_t key[MAXW], u[MAXW];
 #pragma unroll
   for (int s = 0; s < MAXW; ++s) {
-    key[s] = __float_as_uint(cut_clamp(v[s]));
+    key[s] = __float_as_uint(cut_clamp(v[s])) & 0x7fffffffu;   // -0 ranks as +0
     u[s] = ok[s] ? cut_units(v[s]) : 0u;
   }
   uint32_t prefix = 0u;   // digits of tau found so far

@@ -841,3 +841,38 @@ def test_window_step_is_attention_mass_and_selection(ops, b, h, n, d, hkv):
         assert np.abs(np.tril(m1[bi, hi]) - r_ref).max() <= MASS_TOL
         exempt += compare_selection(bits_to_bool(st1[bi, hi], nq), r_ref, eta)
     assert exempt <= max(2, nq // 16)
+
+
+@pytest.mark.parametrize("nq,bh", [(128, 3), (512, 2)])
+def test_select_exact_on_dyadic_masses(ops, nq, bh):
+    """Masses that are multiples of 2^-12 (each row sums to exactly 1, many exact ties):
+    every cumulative sum is exact in the kernel's units and in fp64, so the support must
+    equal the oracle's bit for bit with no near-cut exemption.  A few entries are above 1,
+    negative, -0 or NaN: the kernel counts them as clamp(r, 0, 1), NaN as 0."""
+    rng = np.random.default_rng(7 * nq + bh)
+    m = np.zeros((bh, nq, nq), np.float32)
+    for x in range(bh):
+        for q in range(nq):
+            w = rng.random(q + 1) ** 6 + 1e-3          # a few heavy blocks, long light tail
+            m[x, q, : q + 1] = rng.multinomial(4096, w / w.sum()) / 4096.0
+    odd = []
+    for x in range(bh):
+        for q in rng.choice(np.arange(8, nq), 6, replace=False):
+            b = int(rng.integers(0, q + 1))
+            val = [1.5, -0.25, -0.0, np.nan, 1.0, 0.0][len(odd) % 6]
+            m[x, q, b] = val
+            odd.append((x, q, b))
+    clean = np.nan_to_num(np.clip(m, 0.0, 1.0), nan=0.0).astype(np.float64)
+    mass = torch.from_numpy(m).reshape(1, bh, nq, nq).cuda()
+    for eta in (0.5, 0.75, 0.875, 0.9, 0.99):
+        union = ops.new_bitmask(1, bh, nq, "cuda")
+        step = torch.empty_like(union)
+        ops.select_union(mass, union, eta, step_bits=step)
+        torch.cuda.synchronize()
+        got = bits_to_bool(step.cpu().numpy()[0], nq)
+        e32 = float(np.float32(eta))
+        for x in range(bh):
+            want = O.select(clean[x], e32)
+            bad = np.nonzero((got[x] != want).any(axis=1))[0]
+            assert bad.size == 0, f"eta={eta} head {x}: rows {bad[:8].tolist()} differ"
+    assert ops.device_status() == 0
