@@ -414,7 +414,9 @@ def run_e2e(cfg, runner, host_q, host_k, host_v, reps: int):
     """Trajectories through the public API from pinned host buffers.
 
     Every step copies its Q, K, V host->device (prefetched one step ahead on a
-    copy stream) and copies its O device->host; the clock covers everything.
+    copy stream) and copies its O device->host (on a second copy stream, so the
+    two PCIe directions run at once; O is double-buffered); the clock covers
+    everything.
     """
     import torch
     ops, tr = runner.ops, runner.traj
@@ -422,12 +424,15 @@ def run_e2e(cfg, runner, host_q, host_k, host_v, reps: int):
     T = cfg.steps
     shp = (cfg.batch, cfg.heads, cfg.seqlen, cfg.head_dim)
     bufs = [[torch.empty(shp, dtype=torch.bfloat16, device=dev) for _ in range(3)] for _ in range(2)]
-    obuf = torch.empty(shp, dtype=torch.bfloat16, device=dev)
+    obufs = [torch.empty(shp, dtype=torch.bfloat16, device=dev) for _ in range(2)]
     host_o = torch.empty((T,) + shp, dtype=torch.bfloat16).pin_memory()
     copy = torch.cuda.Stream(device=dev)
+    back = torch.cuda.Stream(device=dev)
     comp = torch.cuda.current_stream(dev)
     ready = [torch.cuda.Event() for _ in range(2)]
     free = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]     # step's O written
+    drained = [torch.cuda.Event() for _ in range(2)]  # O buffer copied out
 
     def h2d(t):
         s = (t - 1) % 2
@@ -436,6 +441,9 @@ def run_e2e(cfg, runner, host_q, host_k, host_v, reps: int):
             for dst, src in zip(bufs[s], (host_q, host_k, host_v)):
                 dst.copy_(src[t - 1], non_blocking=True)
             ready[s].record(copy)
+
+    for s in range(2):   # once: afterwards each refers to its buffer's last copy-out
+        drained[s].record(comp)
 
     def one():
         tr.reset()
@@ -447,10 +455,15 @@ def run_e2e(cfg, runner, host_q, host_k, host_v, reps: int):
             if t < T:
                 h2d(t + 1)
             comp.wait_event(ready[s])
+            comp.wait_event(drained[s])
             qt, kt, vt = bufs[s]
-            tr.step(t, qt, kt, vt, o=obuf)
+            tr.step(t, qt, kt, vt, o=obufs[s])
             free[s].record(comp)
-            host_o[t - 1].copy_(obuf, non_blocking=True)
+            done[s].record(comp)
+            with torch.cuda.stream(back):
+                back.wait_event(done[s])
+                host_o[t - 1].copy_(obufs[s], non_blocking=True)
+                drained[s].record(back)
 
     one()
     torch.cuda.synchronize()
