@@ -98,6 +98,33 @@ def test_null_and_alignment_rejected(lib):
     assert "eta" in lib.last_error()
 
 
+def test_window_step_checks(lib):
+    """wise_window_step validates before enqueueing anything: every pointer but step_bits is
+    required, eta must be > 0, buffers 16-byte aligned, the workspace large enough."""
+    L = lib.lib
+    s = shape(lib)
+    a, ws = 1 << 20, L.wise_mass_workspace_bytes(s)
+    args = [a, a, a, a, a, a, a, None, 0.95, a, ws]
+    assert L.wise_window_step(*args, lib.WiseShape(1, 2, 100, 64, 0.0, 0), None) == \
+        lib.WISE_ERR_SHAPE
+    for i in (0, 1, 2, 3, 4, 5, 6, 9):          # q k v o lse mass union workspace
+        bad = list(args)
+        bad[i] = None
+        assert L.wise_window_step(*bad, s, None) == lib.WISE_ERR_ARG, i
+    for eta in (0.0, -0.5, float("nan")):
+        bad = list(args)
+        bad[8] = eta
+        assert L.wise_window_step(*bad, s, None) == lib.WISE_ERR_ARG
+    assert "eta" in lib.last_error()
+    for i in (0, 3, 4, 5, 9):                  # q, o, lse, mass, workspace misaligned
+        bad = list(args)
+        bad[i] = a + 4
+        assert L.wise_window_step(*bad, s, None) == lib.WISE_ERR_ALIGN, i
+    bad = list(args)
+    bad[10] = ws - 16
+    assert L.wise_window_step(*bad, s, None) == lib.WISE_ERR_WORKSPACE
+
+
 
 def test_select_blocks_checks(lib):
     L = lib.lib
