@@ -15,8 +15,9 @@
 // per key block: rows 4 l .. 4 l + 3 of the group's first and second 128 rows), then
 // the eight lanes holding one query block's 32 rows sum them with three shuffles.
 // Items are numbered group by group, so every warp of the grid has the same short
-// chain of work and the whole causal triangle's loads are in flight at once.  Only
-// admissible (row block, key block) pairs are read or written.
+// chain of work (one round of loads) and the grid streams the causal triangle in about
+// two waves of resident warps at 4K.  Only admissible (row block, key block) pairs are
+// read or written.
 
 #include <cstdint>
 
