@@ -194,6 +194,11 @@ int wise_select_union_blocks(const float* mass, uint32_t* union_bits, uint32_t* 
  *   lse is the natural-log lse of wise_full_attn_mass.
  *   q, k : bf16 [B, H, n, d] (k: [B, kv_heads, n, d]), 16-byte aligned;
  *   lse  : fp32 [B, H, n];  mass16 : fp32 [B, H, n16, n16] output.
+ * wise_full_attn_mass_b16: wise_full_attn_mass (o, lse) plus the same mass16 in one pass:
+ *   the attention kernel records every row's log-sum-exp over each 16-key half block in
+ *   `workspace` (wise_mass_b16_workspace_bytes(shape) bytes, 16-byte aligned) and a
+ *   light kernel averages 2^(blse - lse) over each block's 16 rows; no QK^T recompute.
+ *   All pointers required.
  * wise_select_union_b16: wise_select_union over 16-token blocks: mass16 as above,
  *   union16 / step16 uint32 [B, H, n16, W16] (same bit layout, OR-accumulated /
  *   overwritten), same ranking, cut and eta rules.
@@ -213,6 +218,11 @@ int wise_select_union_blocks(const float* mass, uint32_t* union_bits, uint32_t* 
  */
 int wise_block_mass_b16(const void* q, const void* k, const float* lse, float* mass16,
                         wise_shape_t shape, void* stream);
+int wise_full_attn_mass_b16(const void* q, const void* k, const void* v, void* o, float* lse,
+                            float* mass16, void* workspace, size_t workspace_bytes,
+                            wise_shape_t shape, void* stream);
+/* Workspace bytes of wise_full_attn_mass_b16: B * H * (2 nq) * n * 4. */
+size_t wise_mass_b16_workspace_bytes(wise_shape_t shape);
 int wise_select_union_b16(const float* mass16, uint32_t* union16, uint32_t* step16, float eta,
                           wise_shape_t shape, void* stream);
 size_t wise_schedule_b16_workspace_bytes(wise_shape_t shape);

@@ -54,6 +54,9 @@ _SIGNATURES = {
     "wise_select_union_blocks": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_float, ctypes.c_int32,
                                                 WiseShape, _vp]),
     "wise_block_mass_b16": (ctypes.c_int, [_vp, _vp, _vp, _vp, WiseShape, _vp]),
+    "wise_full_attn_mass_b16": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                               ctypes.c_size_t, WiseShape, _vp]),
+    "wise_mass_b16_workspace_bytes": (ctypes.c_size_t, [WiseShape]),
     "wise_select_union_b16": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_float, WiseShape, _vp]),
     "wise_schedule_b16_workspace_bytes": (ctypes.c_size_t, [WiseShape]),
     "wise_build_schedule_b16": (ctypes.c_int, [_vp, _vp, _vp, _vp, ctypes.c_int64,

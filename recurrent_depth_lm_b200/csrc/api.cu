@@ -447,6 +447,36 @@ int wise_block_mass_b16(const void* q, const void* k, const float* lse, float* m
   return ok();
 }
 
+size_t wise_mass_b16_workspace_bytes(wise_shape_t shape) {
+  return 2 * wise_mass_workspace_bytes(shape);
+}
+
+int wise_full_attn_mass_b16(const void* q, const void* k, const void* v, void* o, float* lse,
+                            float* mass16, void* workspace, size_t workspace_bytes,
+                            wise_shape_t shape, void* stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !lse || !mass16 || !workspace)
+    return fail(WISE_ERR_ARG, "q, k, v, o, lse, mass16 and workspace must be non-NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(WISE_ERR_ALIGN, "q, k, v, o must be 16-byte aligned");
+  if (!aligned16(lse) || !aligned16(mass16) || !aligned16(workspace))
+    return fail(WISE_ERR_ALIGN, "lse, mass16 and workspace must be 16-byte aligned");
+  const size_t need = wise_mass_b16_workspace_bytes(shape);
+  if (workspace_bytes < need)
+    return fail(WISE_ERR_WORKSPACE, "16-token mass workspace of %zu bytes required", need);
+  wise::AttnParams p{};
+  p.lse = lse;
+  p.blse = static_cast<float*>(workspace);
+  p.fine16 = 1;
+  rc = launch_attn(wise::kModeDense, q, k, v, o, p, shape, stream);
+  if (rc) return rc;
+  cudaError_t e = wise::launch_block_mass16(p.blse, lse, mass16, shape.batch * shape.heads,
+                                            shape.seqlen, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "mass16 launch");
+  return ok();
+}
+
 int wise_select_union_b16(const float* mass16, uint32_t* union16, uint32_t* step16, float eta,
                           wise_shape_t shape, void* stream) {
   int rc = check_shape(shape);

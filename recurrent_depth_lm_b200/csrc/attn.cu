@@ -903,18 +903,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;  // all scores -inf then
             const uint64_t nm2 = f2(neg_m, neg_m);
-            uint64_t rs2[2] = {0ull, 0ull};
+            // Dense mode keeps the row sum of each 16-column half apart (the 16-token block
+            // log-sum-exps); the 16-token sparse mode sums the same way, so that on an
+            // all-blocks schedule it reproduces dense attention bit for bit; the 32-token
+            // sparse mode needs only the block's sum.
+            constexpr bool kHalves = MODE == kModeDense || MODE == kModeSparse16;
+            uint64_t rs2[2][2] = {{0ull, 0ull}, {0ull, 0ull}};   // [16-column half][pair parity]
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
               float t0, t1;
               f2_split(fma2(f2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), sc2, nm2), t0, t1);
               const float e0 = fast_exp2(t0), e1 = fast_exp2(t1);
-              rs2[(c >> 1) & 1] = add2(rs2[(c >> 1) & 1], f2(e0, e1));
+              uint64_t& acc = rs2[kHalves ? (c >> 4) : 0][(c >> 1) & 1];
+              acc = add2(acc, f2(e0, e1));
               w[c >> 1] = pack_bf16x2(e0, e1);
             }
-            float lo, hi;
-            f2_split(add2(rs2[0], rs2[1]), lo, hi);
-            const float ps = lo + hi;
+            float ps16[2] = {0.f, 0.f};   // sums over columns 0..15 and 16..31 (dense mode)
+            float ps;
+            {
+              float a0, a1;
+              f2_split(add2(rs2[0][0], rs2[0][1]), a0, a1);
+              if (kHalves) {
+                float b0, b1;
+                f2_split(add2(rs2[1][0], rs2[1][1]), b0, b1);
+                ps16[0] = a0 + a1;
+                ps16[1] = b0 + b1;
+                ps = ps16[0] + ps16[1];
+              } else {
+                ps = a0 + a1;
+              }
+            }
             rs += ps;
             {
               // the block's largest P, computed as its element was, and its bf16 rounding
@@ -925,9 +943,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               // block log-sum-exp of this row over key block kb, log2 domain:
               // blse = m + log2(sum_j 2^(s_ij*scale*log2e - m)); the mass pass turns it
               // into block mass with the final lse.  Layout [bh][key block][row]: 32
-              // lanes store 32 consecutive floats.
-              p.blse[((long long)bh * p.nq + e.kb[s]) * p.n + i] =
-                  ps > 0.f ? m_ref + __log2f(ps) : -INFINITY;
+              // lanes store 32 consecutive floats.  fine16: one value per 16-key half,
+              // key block 2 kb + half of the 16-token blocks.
+              if (p.fine16) {
+                float* dst = p.blse + ((long long)bh * 2 * p.nq + 2 * e.kb[s]) * p.n + i;
+                dst[0] = ps16[0] > 0.f ? m_ref + __log2f(ps16[0]) : -INFINITY;
+                dst[p.n] = ps16[1] > 0.f ? m_ref + __log2f(ps16[1]) : -INFINITY;
+              } else {
+                p.blse[((long long)bh * p.nq + e.kb[s]) * p.n + i] =
+                    ps > 0.f ? m_ref + __log2f(ps) : -INFINITY;
+              }
             }
           } else {
 #pragma unroll

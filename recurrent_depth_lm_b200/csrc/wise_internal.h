@@ -24,7 +24,8 @@ struct AttnParams {
   float* lse;           // [BH, n] output (dense / sparse), nullable
   const float* lse_in;  // [BH, n] input (mass mode)
   float* mass;          // [BH, nq, nq] output (mass mode); [BH, 2nq, 2nq] when fine16
-  int fine16;           // mass mode: block mass of 16-token blocks
+  int fine16;           // mass mode: block mass of 16-token blocks; dense mode with blse:
+                        // one blse per 16-key half ([BH, 2nq, n])
   float* blse;          // [BH, nq, n] block log2-sum-exp side output (dense mode), nullable
   const int32_t* row_offsets;  // sparse mode
   const int32_t* col_idx;      // sparse mode
@@ -43,6 +44,10 @@ int attention_smem_bytes(int mode, int d);
 // Block mass from the recorded per-(row, key block) log-sum-exps.
 cudaError_t launch_block_mass(const float* blse, const float* lse, float* mass, int BH, int n,
                               cudaStream_t stream);
+// The same at 16-token blocks: blse16 is [BH, 2nq, n], mass16 [BH, 2nq, 2nq]; for b > q it
+// writes the diagonal 32-block's entry (0) and nothing else.
+cudaError_t launch_block_mass16(const float* blse16, const float* lse, float* mass16, int BH,
+                                int n, cudaStream_t stream);
 
 cudaError_t launch_select_union(const float* mass, uint32_t* union_bits, uint32_t* step_bits,
                                 float eta, int BH, int nq, cudaStream_t stream);

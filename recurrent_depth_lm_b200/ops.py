@@ -227,6 +227,32 @@ def block_mass_b16(q, k, lse, *, out=None, scale=None, stream=None):
     return out
 
 
+def mass_b16_workspace(b: int, h: int, n: int, head_dim: int, device) -> torch.Tensor:
+    nbytes = lib.wise_mass_b16_workspace_bytes(WiseShape(b, h, n, head_dim, 0.0))
+    return torch.empty(max(1, nbytes // 4), dtype=torch.float32, device=device)
+
+
+def full_attn_mass_b16(q, k, v, *, o=None, lse=None, mass16=None, workspace=None, scale=None,
+                       stream=None):
+    """Dense causal attention plus the 16-token block mass in one pass.  Returns
+    (o, lse, mass16); the mass equals block_mass_b16's without recomputing QK^T."""
+    b, h, n, d = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    kv = _check_qkv(q, k, v, o)
+    if lse is None:
+        lse = torch.empty(b, h, n, dtype=torch.float32, device=q.device)
+    if mass16 is None:
+        mass16 = torch.empty(b, h, n // 16, n // 16, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = mass_b16_workspace(b, h, n, d, q.device)
+    rc = lib.wise_full_attn_mass_b16(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(mass16),
+                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     shape_of(q, scale, kv), _stream(stream))
+    check(rc, "wise_full_attn_mass_b16")
+    return o, lse, mass16
+
+
 def new_bitmask_b16(b: int, h: int, n: int, device) -> torch.Tensor:
     """Zeroed 16-token working-set masks [B, H, n/16, ceil(n/16/32)]."""
     return new_bitmask(b, h, n // 16, device)

@@ -60,6 +60,8 @@ class WiseTrajectory:
             self.mass16 = torch.empty(batch, heads, seqlen // 16, seqlen // 16,
                                       dtype=torch.float32, device=dev)
             self.union = ops.new_bitmask_b16(batch, heads, seqlen, dev)
+            # per-(row, 16-key block) log-sum-exps of the one-pass 16-token mass
+            self.mass_ws = ops.mass_b16_workspace(batch, heads, seqlen, head_dim, dev)
         else:
             self.mass = torch.empty(batch, heads, self.nq, self.nq, dtype=torch.float32,
                                     device=dev)
@@ -108,10 +110,9 @@ class WiseTrajectory:
         if t <= self.t_d:
             first = t == 1 and self.mass1 is not None   # step-1 masses for the controls
             if self.block == 16 and self.in_window(t):
-                o, _, _ = ops.full_attn_mass(q, k, v, o=o, lse=self.lse, scale=self.scale,
-                                             stream=stream)
-                ops.block_mass_b16(q, k, self.lse, out=self.mass16, scale=self.scale,
-                                   stream=stream)
+                o, _, _ = ops.full_attn_mass_b16(q, k, v, o=o, lse=self.lse, mass16=self.mass16,
+                                                 workspace=self.mass_ws, scale=self.scale,
+                                                 stream=stream)
                 sb = None
                 if self.keep_step_bits:
                     sb = torch.empty_like(self.union)

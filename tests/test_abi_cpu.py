@@ -98,6 +98,27 @@ def test_null_and_alignment_rejected(lib):
     assert "eta" in lib.last_error()
 
 
+def test_full_attn_mass_b16_checks(lib):
+    L = lib.lib
+    s = shape(lib)
+    a, ws = 1 << 20, L.wise_mass_b16_workspace_bytes(s)
+    assert ws == 2 * L.wise_mass_workspace_bytes(s)
+    args = [a, a, a, a, a, a, a, ws]
+    for i in range(7):                          # q k v o lse mass16 workspace
+        bad = list(args)
+        bad[i] = None
+        assert L.wise_full_attn_mass_b16(*bad, s, None) == lib.WISE_ERR_ARG, i
+    for i in (0, 3, 4, 5, 6):
+        bad = list(args)
+        bad[i] = a + 4
+        assert L.wise_full_attn_mass_b16(*bad, s, None) == lib.WISE_ERR_ALIGN, i
+    bad = list(args)
+    bad[7] = ws - 16
+    assert L.wise_full_attn_mass_b16(*bad, s, None) == lib.WISE_ERR_WORKSPACE
+    assert L.wise_full_attn_mass_b16(*args, lib.WiseShape(1, 2, 100, 64, 0.0, 0), None) == \
+        lib.WISE_ERR_SHAPE
+
+
 def test_window_step_checks(lib):
     """wise_window_step validates before enqueueing anything: every pointer but step_bits is
     required, eta must be > 0, buffers 16-byte aligned, the workspace large enough."""
